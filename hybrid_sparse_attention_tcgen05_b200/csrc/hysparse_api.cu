@@ -1,0 +1,226 @@
+// C-ABI entry points of libhysparse.so: argument checks on the host, the
+// workspace layout, and dispatch to the kernels.  See include/hysparse.h for
+// the contract of every call.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "hysparse.h"
+#include "internal.h"
+
+namespace hs {
+namespace {
+
+constexpr int kMaxTopk = 4096;
+constexpr int kMaxWindow = 1024;
+constexpr int kMaxGroup = 32;
+constexpr int kMaxLen = 1 << 24;
+
+bool aligned16(const void *p) { return p != nullptr && ((uintptr_t)p & 15u) == 0; }
+
+int resolve_shape(const hs_shape *in, Shape *out) {
+    if (in == nullptr) return HS_ERR_INVALID_ARG;
+    const hs_shape &s = *in;
+    if (s.B < 1 || s.Lq < 1 || s.Lkv < 1 || s.Hq < 1 || s.Hkv < 1 || s.d < 1) return HS_ERR_INVALID_ARG;
+    if (s.Lq > s.Lkv || s.Lkv > kMaxLen || s.Hq % s.Hkv != 0) return HS_ERR_INVALID_ARG;
+    if (s.Hq / s.Hkv > kMaxGroup) return HS_ERR_UNSUPPORTED;
+    if (s.dtype != HS_F32 && s.dtype != HS_BF16) return HS_ERR_INVALID_ARG;
+    const bool ok = (s.dtype == HS_F32 && (s.d == 64 || s.d == 128)) || (s.dtype == HS_BF16 && s.d == 128);
+    if (!ok) return HS_ERR_UNSUPPORTED;
+    if (!(s.scale == s.scale) || isinf(s.scale)) return HS_ERR_INVALID_ARG;
+    *out = Shape{s.B, s.Lq, s.Lkv, s.Hq, s.Hkv, s.d, s.dtype,
+                 s.scale > 0.f ? s.scale : 1.0f / sqrtf((float)s.d)};
+    return HS_OK;
+}
+
+// Workspace regions (byte offsets), all 256-byte aligned.
+struct WsLayout {
+    size_t status = 0;
+    size_t stats = 0, stats_end = 0;          // full layer per-row statistics
+    size_t block_scores = 0, block_lse = 0, block_idx = 0;
+    size_t total = 0;
+};
+
+WsLayout ws_layout(const Shape &s, int topk, int row_chunk) {
+    WsLayout L;
+    size_t off = kStatusBytes;
+    L.stats = off;
+    off = align_up(off + (size_t)s.B * s.Hq * s.Lq * 2 * sizeof(float), 256);
+    L.stats_end = off;
+    const int chunk = (row_chunk <= 0 || row_chunk > s.Lq) ? s.Lq : row_chunk;
+    L.block_scores = off;
+    off = align_up(off + (size_t)s.B * s.Hkv * chunk * (size_t)s.Lkv * sizeof(float), 256);
+    L.block_lse = off;
+    off = align_up(off + (size_t)s.B * s.Hq * s.Lq * sizeof(float), 256);
+    L.block_idx = off;
+    off = align_up(off + (size_t)s.B * s.Hkv * s.Lq * (size_t)topk * sizeof(int32_t), 256);
+    L.total = off;
+    return L;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? HS_OK : HS_ERR_CUDA; }
+
+int check_full_args(const Shape &s, const void *q, const void *k, const void *v, void *out,
+                    float *lse, float *scores, long long ld, int row_begin, int row_count) {
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+        return HS_ERR_INVALID_ARG;
+    if (row_begin < 0 || row_count < 1 || row_begin > s.Lq - row_count) return HS_ERR_INVALID_ARG;
+    if (scores != nullptr && (!aligned16(scores) || ld < s.Lkv)) return HS_ERR_INVALID_ARG;
+    return HS_OK;
+}
+
+int run_full(const Shape &s, const void *q, const void *k, const void *v, void *out, float *lse,
+             float *scores, long long ld, int row_begin, int row_count, void *ws, cudaStream_t st) {
+    (void)ws;
+    return cuda_status(full_attn_scores_simt_launch(s, q, k, v, out, lse, scores, ld, row_begin,
+                                                    row_count, st));
+}
+
+int run_topk(const Shape &s, const float *scores, long long ld, int row_begin, int row_count,
+             int topk, int32_t *idx, cudaStream_t st) {
+    return cuda_status(topk_launch(s, scores, ld, row_begin, row_count, topk, idx, st));
+}
+
+int run_sparse(const Shape &s, const void *q, const void *k, const void *v, const int32_t *idx,
+               int topk, const float *gate, int window, void *out, void *og, void *ol, void *ws,
+               cudaStream_t st) {
+    unsigned int *status = reinterpret_cast<unsigned int *>(ws);
+    return cuda_status(sparse_attn_simt_launch(s, q, k, v, idx, topk, gate, window, out, og, ol,
+                                               status, st));
+}
+
+}  // namespace
+}  // namespace hs
+
+using namespace hs;
+
+extern "C" {
+
+size_t hysparse_workspace_size(const hs_shape *shape, int topk, int window, int n_sparse,
+                               int row_chunk) {
+    Shape s;
+    if (resolve_shape(shape, &s) != HS_OK) return 0;
+    if (topk < 1 || topk > kMaxTopk || window < 1 || window > kMaxWindow || n_sparse < 0) return 0;
+    return ws_layout(s, topk, row_chunk).total;
+}
+
+int hysparse_full_attn_scores(const hs_shape *shape, const void *q, const void *k, const void *v,
+                              void *out, float *lse, float *scores, long long ld_scores,
+                              int row_begin, int row_count, void *ws, size_t ws_bytes,
+                              hs_stream_t stream) {
+    Shape s;
+    int rc = resolve_shape(shape, &s);
+    if (rc != HS_OK) return rc;
+    rc = check_full_args(s, q, k, v, out, lse, scores, ld_scores, row_begin, row_count);
+    if (rc != HS_OK) return rc;
+    if (!aligned16(ws)) return HS_ERR_INVALID_ARG;
+    if (ws_bytes < ws_layout(s, 1, row_count).stats_end) return HS_ERR_WORKSPACE;
+    return run_full(s, q, k, v, out, lse, scores, ld_scores, row_begin, row_count, ws,
+                    (cudaStream_t)stream);
+}
+
+int hysparse_topk(const hs_shape *shape, const float *scores, long long ld_scores, int row_begin,
+                  int row_count, int topk, int32_t *idx, hs_stream_t stream) {
+    Shape s;
+    int rc = resolve_shape(shape, &s);
+    if (rc != HS_OK) return rc;
+    if (!aligned16(scores) || !aligned16(idx) || ld_scores < s.Lkv) return HS_ERR_INVALID_ARG;
+    if (row_begin < 0 || row_count < 1 || row_begin > s.Lq - row_count) return HS_ERR_INVALID_ARG;
+    if (topk < 1 || topk > kMaxTopk) return HS_ERR_INVALID_ARG;
+    return run_topk(s, scores, ld_scores, row_begin, row_count, topk, idx, (cudaStream_t)stream);
+}
+
+int hysparse_sparse_attn(const hs_shape *shape, const void *q, const void *k, const void *v,
+                         const int32_t *idx, int topk, const float *gate_logit, int window,
+                         void *out, void *out_global, void *out_local, void *ws, size_t ws_bytes,
+                         hs_stream_t stream) {
+    Shape s;
+    int rc = resolve_shape(shape, &s);
+    if (rc != HS_OK) return rc;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) ||
+        !aligned16(gate_logit) || !aligned16(out))
+        return HS_ERR_INVALID_ARG;
+    if ((out_global && !aligned16(out_global)) || (out_local && !aligned16(out_local)))
+        return HS_ERR_INVALID_ARG;
+    if (topk < 1 || topk > kMaxTopk || window < 1 || window > kMaxWindow) return HS_ERR_INVALID_ARG;
+    if (!aligned16(ws)) return HS_ERR_INVALID_ARG;
+    if (ws_bytes < ws_layout(s, topk, 1).stats_end) return HS_ERR_WORKSPACE;
+    return run_sparse(s, q, k, v, idx, topk, gate_logit, window, out, out_global, out_local, ws,
+                      (cudaStream_t)stream);
+}
+
+int hysparse_block(const hs_shape *shape, const void *q_full, const void *k, const void *v,
+                   void *out_full, float *lse, int n_sparse, const void *const *q_sparse,
+                   const float *const *gate_logit, void *const *out_sparse, int topk, int window,
+                   int32_t *idx_out, int row_chunk, void *ws, size_t ws_bytes,
+                   hs_stream_t stream) {
+    Shape s;
+    int rc = resolve_shape(shape, &s);
+    if (rc != HS_OK) return rc;
+    if (topk < 1 || topk > kMaxTopk || window < 1 || window > kMaxWindow || n_sparse < 0)
+        return HS_ERR_INVALID_ARG;
+    if (n_sparse > 0 && (q_sparse == nullptr || gate_logit == nullptr || out_sparse == nullptr))
+        return HS_ERR_INVALID_ARG;
+    if (!aligned16(q_full) || !aligned16(k) || !aligned16(v) || !aligned16(out_full))
+        return HS_ERR_INVALID_ARG;
+    if ((lse && !aligned16(lse)) || (idx_out && !aligned16(idx_out))) return HS_ERR_INVALID_ARG;
+    for (int n = 0; n < n_sparse; ++n)
+        if (!aligned16(q_sparse[n]) || !aligned16(gate_logit[n]) || !aligned16(out_sparse[n]))
+            return HS_ERR_INVALID_ARG;
+    if (!aligned16(ws)) return HS_ERR_INVALID_ARG;
+    const int chunk = (row_chunk <= 0 || row_chunk > s.Lq) ? s.Lq : row_chunk;
+    const WsLayout L = ws_layout(s, topk, chunk);
+    if (ws_bytes < L.total) return HS_ERR_WORKSPACE;
+
+    char *w = reinterpret_cast<char *>(ws);
+    float *scores = reinterpret_cast<float *>(w + L.block_scores);
+    float *lse_buf = lse ? lse : reinterpret_cast<float *>(w + L.block_lse);
+    int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(w + L.block_idx);
+    cudaStream_t st = (cudaStream_t)stream;
+    for (int r0 = 0; r0 < s.Lq; r0 += chunk) {
+        const int rows = (s.Lq - r0 < chunk) ? s.Lq - r0 : chunk;
+        rc = run_full(s, q_full, k, v, out_full, lse_buf, scores, s.Lkv, r0, rows, ws, st);
+        if (rc != HS_OK) return rc;
+        rc = run_topk(s, scores, s.Lkv, r0, rows, topk, idx, st);
+        if (rc != HS_OK) return rc;
+    }
+    for (int n = 0; n < n_sparse; ++n) {
+        rc = run_sparse(s, q_sparse[n], k, v, idx, topk, gate_logit[n], window, out_sparse[n],
+                        nullptr, nullptr, ws, st);
+        if (rc != HS_OK) return rc;
+    }
+    return HS_OK;
+}
+
+int hysparse_workspace_status(void *ws, hs_stream_t stream) {
+    if (!aligned16(ws)) return HS_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    unsigned int word = 0;
+    if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return HS_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return HS_ERR_CUDA;
+    if (word == 0) return HS_OK;
+    if (cudaMemsetAsync(ws, 0, sizeof(word), st) != cudaSuccess) return HS_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return HS_ERR_CUDA;
+    for (int c = 1; c < 32; ++c)
+        if (word & (1u << c)) return c;
+    return HS_ERR_CUDA;
+}
+
+const char *hysparse_status_string(int status) {
+    switch (status) {
+        case HS_OK: return "ok";
+        case HS_ERR_INVALID_ARG: return "invalid argument";
+        case HS_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case HS_ERR_WORKSPACE: return "workspace too small";
+        case HS_ERR_CUDA: return "CUDA error";
+        case HS_ERR_INVALID_INDEX: return "index list entry outside [-1, pos]";
+        case HS_ERR_TIMEOUT: return "bounded wait in a kernel timed out";
+        default: return "unknown status";
+    }
+}
+
+const char *hysparse_version(void) { return "hysparse-b200 0.1"; }
+
+}  // extern "C"

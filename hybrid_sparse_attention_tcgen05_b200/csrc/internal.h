@@ -1,0 +1,34 @@
+// Internal launcher interface between the C-ABI layer (hysparse_api.cu) and
+// the kernel files.  Not installed, not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hysparse.h"
+
+namespace hs {
+
+// A validated hs_shape (scale resolved).
+struct Shape {
+    int B, Lq, Lkv, Hq, Hkv, d;
+    int dtype;
+    float scale;
+    int G() const { return Hq / Hkv; }
+};
+
+// simt_attn.cu
+cudaError_t full_attn_scores_simt_launch(const Shape &s, const void *q, const void *k,
+                                         const void *v, void *out, float *lse, float *scores,
+                                         long long ld, int row_begin, int row_count,
+                                         cudaStream_t st);
+cudaError_t sparse_attn_simt_launch(const Shape &s, const void *q, const void *k, const void *v,
+                                    const int32_t *idx, int topk, const float *gate, int window,
+                                    void *out, void *og, void *ol, unsigned int *status,
+                                    cudaStream_t st);
+
+// topk.cu
+cudaError_t topk_launch(const Shape &s, const float *scores, long long ld, int row_begin,
+                        int row_count, int topk, int32_t *idx, cudaStream_t st);
+
+}  // namespace hs

@@ -1,0 +1,161 @@
+/*
+ * hysparse.h -- C ABI of libhysparse.so, the B200 (sm_100a) hot path of the
+ * HySparse hybrid block.
+ *
+ * Method (HySparse: A Hybrid Sparse Attention Architecture with Oracle Token
+ * Selection and KV Cache Sharing, abstract; intelliparadigm write-up, sections
+ * 2.1 "hybrid block", 2.2 "dual-branch sparse attention", 3.1 "cross-layer
+ * sharing"): a full causal attention layer is followed by N sparse layers.
+ * The full layer is the only writer of the KV cache and the "oracle" of token
+ * importance; each sparse layer reuses its KV cache and its top-k key set and
+ * mixes a global branch over those keys with a 128-token local window through
+ * a sigmoid gate.
+ *
+ * Notation used below:
+ *   B batch, Lq query rows, Lkv cache length, Hq query heads, Hkv KV heads,
+ *   d head dim, G = Hq / Hkv (query head h reads KV head h / G),
+ *   pos(i) = Lkv - Lq + i  (causal, bottom-right aligned: row i sees keys
+ *   0 .. pos(i); decode is Lq = 1 with the new token at Lkv - 1).
+ *
+ * Layouts (row-major, contiguous, every pointer 16-byte aligned):
+ *   q, q_sparse[n], out, out_sparse[n]  [B][Lq][Hq][d]   (dtype of the shape)
+ *   k, v                               [B][Lkv][Hkv][d]  (dtype of the shape)
+ *   lse                                [B][Hq][Lq]        float, natural log
+ *   scores (one row chunk)             [B][Hkv][row_count][ld_scores] float
+ *   idx                                [B][Hkv][Lq][topk] int32
+ *   gate_logit                         [B][Lq][Hq]        float
+ *
+ * Conventions for every entry point:
+ *   - All device buffers are owned by the caller (e.g. allocated by PyTorch).
+ *     The library allocates no device or host memory and keeps no state
+ *     between calls; scratch lives in the caller's workspace `ws`.
+ *   - Work is enqueued on `stream` and is asynchronous; nothing synchronises
+ *     except hysparse_workspace_status.
+ *   - Arguments are checked on the host before anything is launched; a
+ *     non-zero return means nothing was launched and no output was touched.
+ *     A failed launch returns HS_ERR_CUDA.
+ *   - Supported: dtype HS_F32 with d in {64, 128}; dtype HS_BF16 with
+ *     d = 128; Hq % Hkv == 0; 1 <= Hq / Hkv <= 32; Lq <= Lkv;
+ *     1 <= topk <= 4096; 1 <= window <= 1024.
+ *   - NaN or Inf inputs give undefined (but memory-safe) results.
+ */
+#ifndef HYSPARSE_H
+#define HYSPARSE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream; NULL is the legacy default stream. */
+typedef struct CUstream_st *hs_stream_t;
+
+typedef enum {
+    HS_OK = 0,
+    HS_ERR_INVALID_ARG = 1,   /* null or misaligned pointer, bad size, bad shape */
+    HS_ERR_UNSUPPORTED = 2,   /* valid but not implemented (dtype/d combination) */
+    HS_ERR_WORKSPACE = 3,     /* ws_bytes below hysparse_workspace_size() */
+    HS_ERR_CUDA = 4,          /* a CUDA call or kernel launch failed */
+    HS_ERR_INVALID_INDEX = 5, /* (device) an index list entry outside [-1, pos] */
+    HS_ERR_TIMEOUT = 6        /* (device) a bounded wait inside a kernel gave up */
+} hs_status;
+
+typedef enum { HS_F32 = 0, HS_BF16 = 1 } hs_dtype;
+
+typedef struct {
+    int B, Lq, Lkv, Hq, Hkv, d;
+    int dtype;    /* hs_dtype */
+    float scale;  /* softmax scale on q.k; <= 0 selects 1/sqrt(d) */
+} hs_shape;
+
+/* Bytes of device workspace that hysparse_full_attn_scores,
+ * hysparse_sparse_attn and hysparse_block need for this shape.  `row_chunk`
+ * is the number of query rows hysparse_block scores at a time (<= 0: all Lq
+ * rows); the other arguments are those of the calls.  Returns 0 for an
+ * invalid shape.  The first 256 bytes of a workspace hold a status word (see
+ * hysparse_workspace_status); zero them once before first use (the calls
+ * only ever OR error bits into it). */
+size_t hysparse_workspace_size(const hs_shape *shape, int topk, int window, int n_sparse,
+                               int row_chunk);
+
+/* The full attention layer of the hybrid block, restricted to the query rows
+ * [row_begin, row_begin + row_count) of every batch element.
+ *
+ * Computes (HySparse abstract; write-up section 2.1, the full layer as the
+ * token-importance oracle; the score is the group sum of the softmax
+ * probabilities over the query heads that share a KV head):
+ *   out[b,i,h]  = sum_{j <= pos(i)} softmax_j(scale * q[b,i,h].k[b,j,h/G]) v[b,j,h/G]
+ *   lse[b,h,i]  = ln sum_{j <= pos(i)} exp(scale * q[b,i,h].k[b,j,h/G])
+ *   scores[b,g,i-row_begin,j] = sum_{h : h/G = g} exp(scale * q.k_j - lse[b,h,i])
+ *                              for j <= pos(i); entries j > pos(i) are left
+ *                              unspecified and are never read by hysparse_topk.
+ * `scores` may be NULL (forward pass only); otherwise ld_scores >= Lkv.
+ * Only out/lse entries of the listed rows are written.
+ * Decode (Lq == 1) uses split-K over the cache and needs `ws`.
+ * Errors: HS_ERR_INVALID_ARG, HS_ERR_UNSUPPORTED, HS_ERR_WORKSPACE, HS_ERR_CUDA. */
+int hysparse_full_attn_scores(const hs_shape *shape, const void *q, const void *k, const void *v,
+                              void *out, float *lse, float *scores, long long ld_scores,
+                              int row_begin, int row_count, void *ws, size_t ws_bytes,
+                              hs_stream_t stream);
+
+/* Per-row top-k over one chunk of importance rows (write-up section 2.2: the
+ * global branch attends over the full layer's TopK indices; section 3.1: one
+ * index set per row is shared by the following sparse layers).
+ * For every (b, g, i) with i in [row_begin, row_begin + row_count): the
+ * `topk` keys j <= pos(i) with the largest scores[b,g,i-row_begin,j], ties
+ * going to the lower j.  A row with pos(i) + 1 <= topk takes all its keys.
+ * The set is written to idx[b,g,i,:] in ascending key order, padded with -1.
+ * Scores must be >= 0 (importance values are).  Exact and deterministic.
+ * Errors: HS_ERR_INVALID_ARG, HS_ERR_CUDA. */
+int hysparse_topk(const hs_shape *shape, const float *scores, long long ld_scores, int row_begin,
+                  int row_count, int topk, int32_t *idx, hs_stream_t stream);
+
+/* One sparse layer (write-up section 2.2, dual-branch sparse attention;
+ * section 3.1, KV cache reuse: reads the full layer's k and v, writes no KV):
+ *   Og = softmax attention of q[b,i,h] over { k_j : j in idx[b,h/G,i,:], j != -1 }
+ *   Ol = softmax attention of q[b,i,h] over { k_j : max(0, pos(i)-window+1) <= j <= pos(i) }
+ *   out = sigmoid(gate_logit[b,i,h]) * Og + (1 - sigmoid(gate_logit[b,i,h])) * Ol
+ * The two branches may share keys; each has its own softmax.  An index list
+ * with no valid entry gives Og = 0.  Index lists must hold distinct keys in
+ * [0, pos(i)] (any order) padded with -1; entries outside [-1, pos(i)] are
+ * skipped and reported as HS_ERR_INVALID_INDEX through the workspace status
+ * word.  out_global / out_local (nullable) receive Og and Ol.
+ * Decode (Lq == 1) uses split-K and needs `ws`.
+ * Errors: HS_ERR_INVALID_ARG, HS_ERR_UNSUPPORTED, HS_ERR_WORKSPACE, HS_ERR_CUDA. */
+int hysparse_sparse_attn(const hs_shape *shape, const void *q, const void *k, const void *v,
+                         const int32_t *idx, int topk, const float *gate_logit, int window,
+                         void *out, void *out_global, void *out_local, void *ws, size_t ws_bytes,
+                         hs_stream_t stream);
+
+/* A whole hybrid block (HySparse abstract: one full layer interleaved with
+ * several sparse layers; write-up section 3.1: index sharing and cache reuse):
+ * the full layer over all rows (out_full, and its LSE into `lse` when not
+ * NULL), its importance scores and top-k (scored `row_chunk` rows at a time
+ * inside `ws`), then n_sparse sparse layers, each with its own queries and
+ * gate logits, all reusing k, v and the one index set.
+ * q_sparse, gate_logit and out_sparse are HOST arrays of n_sparse DEVICE
+ * pointers.  idx_out (nullable) receives the index set [B][Hkv][Lq][topk];
+ * when NULL it is kept in `ws`.  Errors: as the calls it makes. */
+int hysparse_block(const hs_shape *shape, const void *q_full, const void *k, const void *v,
+                   void *out_full, float *lse, int n_sparse, const void *const *q_sparse,
+                   const float *const *gate_logit, void *const *out_sparse, int topk, int window,
+                   int32_t *idx_out, int row_chunk, void *ws, size_t ws_bytes, hs_stream_t stream);
+
+/* Synchronises `stream`, reads the workspace status word (HS_OK or the
+ * lowest-numbered device error recorded since it was last cleared), clears
+ * it and returns it.  Returns HS_ERR_CUDA if the synchronisation fails. */
+int hysparse_workspace_status(void *ws, hs_stream_t stream);
+
+/* Static text for a status code. */
+const char *hysparse_status_string(int status);
+
+/* Library version, e.g. "hysparse-b200 0.1". */
+const char *hysparse_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYSPARSE_H */

@@ -1,0 +1,215 @@
+"""GPU (CUDA path, through the C ABI) against the CPU oracle on the same
+seeded inputs.  Needs a B200; run with ``pytest -m gpu``."""
+from __future__ import annotations
+
+import pytest
+import torch
+
+import oracle
+import hybrid_sparse_attention_tcgen05_b200 as hs
+from hybrid_sparse_attention_tcgen05_b200 import inputs as gen
+from parity import (check_out, check_scores, check_topk, gather_idx_rows, gather_rows, rows_for,
+                    scale_of)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def run_stages(inp, w, row_chunk=None):
+    """full_attn_scores (one chunk = all rows unless row_chunk) -> topk ->
+    sparse layers, each through its own C-ABI call."""
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    shape = hs.shape_of(q, k)
+    out = torch.empty_like(q)
+    lse = torch.empty(w.B, w.Hq, w.Lq, dtype=torch.float32, device=DEV)
+    idx = torch.empty(w.B, w.Hkv, w.Lq, w.topk, dtype=torch.int32, device=DEV)
+    chunk = row_chunk or w.Lq
+    scores_all = torch.empty(w.B, w.Hkv, w.Lq, w.Lkv, dtype=torch.float32, device=DEV) \
+        if w.Lq * w.Lkv * w.B * w.Hkv <= (1 << 28) else None
+    for r0 in range(0, w.Lq, chunk):
+        rc = min(chunk, w.Lq - r0)
+        _, _, sc = hs.full_attn_scores(q, k, v, row_begin=r0, row_count=rc, out=out, lse=lse)
+        hs.topk(shape, sc, w.topk, row_begin=r0, idx=idx)
+        if scores_all is not None:
+            scores_all[:, :, r0:r0 + rc] = sc
+    outs = [hs.sparse_attn(qs, k, v, idx, gt, w.window, want_branches=True)
+            for qs, gt in zip(inp["q_sparse"], inp["gate"])]
+    torch.cuda.synchronize()
+    return out, lse, idx, scores_all, outs
+
+
+def oracle_check_rows(inp, w, rows, out, lse, idx, scores_all, outs, check_own_idx=True):
+    """Compare the listed rows against the oracle (full layer, scores, top-k,
+    every sparse layer on the oracle's and on the GPU's own index sets)."""
+    scale = scale_of(w.d)
+    k_h, v_h = inp["k"].to("cpu"), inp["v"].to("cpu")
+    qr = gather_rows(inp["q"], rows)
+    o_out, o_lse, o_sc = oracle.full_rows(qr, k_h, v_h, rows, w.Lq, scale)
+    check_out("full out", gather_rows(out, rows), o_out, w.dtype)
+    b = torch.tensor([r[0] for r in rows])
+    i = torch.tensor([r[1] for r in rows])
+    g_lse = lse.to("cpu")[b, :, i]
+    assert float((g_lse.double() - o_lse).abs().max()) <= 1e-4
+    n_valid = [w.Lkv - w.Lq + r[1] + 1 for r in rows for _ in range(w.Hkv)]
+    if scores_all is not None:
+        g_sc = scores_all.to("cpu")[b, :, i].reshape(-1, w.Lkv)
+        check_scores(g_sc, o_sc.reshape(-1, w.Lkv), n_valid)
+    g_idx = gather_idx_rows(idx, rows)
+    stats = check_topk(g_idx.reshape(-1, w.topk), o_sc.reshape(-1, w.Lkv), n_valid, w.topk)
+    o_idx = oracle.topk_rows(o_sc.reshape(-1, w.Lkv), n_valid, w.topk).reshape(len(rows), w.Hkv, w.topk)
+    for n, (qs, gt) in enumerate(zip(inp["q_sparse"], inp["gate"])):
+        g_out, g_og, g_ol = outs[n]
+        qsr, gtr = gather_rows(qs, rows), gather_rows(gt, rows)
+        # on the GPU's own index sets
+        r_out, r_og, r_ol = oracle.sparse_rows(qsr, k_h, v_h, rows, w.Lq, scale, g_idx, gtr, w.window)
+        check_out(f"sparse{n} out (own idx)", gather_rows(g_out, rows), r_out, w.dtype)
+        check_out(f"sparse{n} global (own idx)", gather_rows(g_og, rows), r_og, w.dtype)
+        check_out(f"sparse{n} local", gather_rows(g_ol, rows), r_ol, w.dtype)
+    return stats, o_idx
+
+
+def sparse_on_indices(inp, w, idx_dev):
+    return [hs.sparse_attn(qs, inp["k"], inp["v"], idx_dev, gt, w.window, want_branches=True)
+            for qs, gt in zip(inp["q_sparse"], inp["gate"])]
+
+
+# ---------------------------------------------------------------- tiny (fp32)
+
+def _tiny_inputs():
+    w = gen.WORKLOADS["tiny"]
+    cpu = gen.make_inputs(w, seed=0, device="cpu")
+    dev = {key: (val.to(DEV) if torch.is_tensor(val) else [x.to(DEV) for x in val])
+           for key, val in cpu.items()}
+    return w, dev
+
+
+def test_tiny_all_rows():
+    w, inp = _tiny_inputs()
+    out, lse, idx, sc, outs = run_stages(inp, w)
+    rows = rows_for(w.B, w.Lq, range(w.Lq))
+    stats, o_idx = oracle_check_rows(inp, w, rows, out, lse, idx, sc, outs)
+    # sparse layer on the oracle's index sets
+    idx_o = torch.empty_like(idx)
+    idx_o[0] = o_idx.permute(1, 0, 2).to(DEV)
+    outs_o = sparse_on_indices(inp, w, idx_o)
+    k_h, v_h = inp["k"].cpu(), inp["v"].cpu()
+    for n, (qs, gt) in enumerate(zip(inp["q_sparse"], inp["gate"])):
+        r_out, r_og, _ = oracle.sparse_rows(gather_rows(qs, rows), k_h, v_h, rows, w.Lq,
+                                            scale_of(w.d), o_idx, gather_rows(gt, rows), w.window)
+        check_out("sparse out (oracle idx)", gather_rows(outs_o[n][0], rows), r_out, w.dtype)
+        check_out("sparse global (oracle idx)", gather_rows(outs_o[n][1], rows), r_og, w.dtype)
+
+
+def test_tiny_block_matches_stages():
+    w, inp = _tiny_inputs()
+    out, lse, idx, _, outs = run_stages(inp, w)
+    for chunk in (0, 100):
+        of, lb, ib, ob = hs.block(inp["q"], inp["k"], inp["v"], inp["q_sparse"], inp["gate"], w.topk,
+                                  w.window, row_chunk=chunk)
+        torch.cuda.synchronize()
+        assert torch.equal(ib, idx)
+        assert torch.equal(of, out)
+        assert torch.equal(lb, lse)
+        for n in range(w.n_sparse):
+            assert torch.equal(ob[n], outs[n][0])
+
+
+def test_topk_stage_isolated_bit_exact():
+    """The same fp32 score buffer through the GPU top-k and the oracle top-k:
+    identical index lists, no tolerance band."""
+    w, inp = _tiny_inputs()
+    _, _, idx, sc, _ = run_stages(inp, w)
+    n_valid = [w.Lkv - w.Lq + i + 1 for i in range(w.Lq)]
+    o_idx = oracle.topk_rows(sc[0, 0].cpu(), n_valid, w.topk)
+    assert torch.equal(idx[0, 0].cpu(), o_idx)
+
+
+@pytest.mark.parametrize("case", ["ties", "all_equal", "zeros_and_denormals", "long_rows"])
+def test_topk_synthetic_rows_bit_exact(case):
+    """Score rows built directly (not by the CUDA path), with exact ties."""
+    g = torch.Generator().manual_seed(7)
+    B, Hkv, Lq, Lkv, k = 2, 3, 37, 300, 29
+    if case == "long_rows":
+        Lq, Lkv, k = 5, 70000, 2048
+    s = torch.rand(B, Hkv, Lq, Lkv, generator=g)
+    if case == "ties":
+        s = torch.round(s * 16) / 16
+    elif case == "all_equal":
+        s[:] = 0.125
+    elif case == "zeros_and_denormals":
+        s = torch.where(s < 0.5, torch.zeros_like(s), s * 1e-39)
+    elif case == "long_rows":
+        s = torch.round(s * 4096) / 4096
+    shape = hs.HsShape(B, Lq, Lkv, 4 * Hkv, Hkv, 128, 1, 0.0)
+    idx = hs.topk(shape, s.to(DEV), k)
+    n_valid = [Lkv - Lq + i + 1 for _ in range(B) for _ in range(Hkv) for i in range(Lq)]
+    o_idx = oracle.topk_rows(s.reshape(-1, Lkv), n_valid, k).reshape(B, Hkv, Lq, k)
+    assert torch.equal(idx.cpu(), o_idx)
+
+
+# ------------------------------------------------------------- shape sweep
+
+SWEEP = [
+    # name, B, Lq, Lkv, Hq, Hkv, d, dtype, topk, window, dist
+    ("f32_ragged", 2, 77, 77, 4, 2, 64, "f32", 9, 5, "normal"),
+    ("f32_chunked_prefix", 1, 40, 150, 8, 1, 128, "f32", 33, 16, "normal"),
+    ("f32_decode", 3, 1, 300, 8, 2, 64, "f32", 64, 128, "normal"),
+    ("f32_topk_ge_len", 1, 50, 50, 2, 2, 64, "f32", 64, 1, "normal"),
+    ("bf16_small", 1, 300, 300, 8, 2, 128, "bf16", 64, 128, "shifted"),
+    ("bf16_g16", 1, 200, 260, 32, 2, 128, "bf16", 100, 17, "shifted"),
+    ("bf16_g1_ragged", 2, 129, 129, 2, 2, 128, "bf16", 1, 3, "normal"),
+    ("bf16_decode", 4, 1, 1000, 32, 8, 128, "bf16", 128, 128, "normal"),
+    ("bf16_window_ge_len", 1, 130, 130, 4, 1, 128, "bf16", 16, 1024, "shifted"),
+]
+
+
+@pytest.mark.parametrize("case", SWEEP, ids=lambda c: c[0])
+def test_shape_sweep_all_rows(case):
+    name, B, Lq, Lkv, Hq, Hkv, d, dt, topk, window, dist = case
+    w = gen.Workload(name, B, Lq, Lkv, Hq, Hkv, d, dt, topk, window, 2, dist)
+    cpu = gen.make_inputs(w, seed=3, device="cpu")
+    inp = {key: (val.to(DEV) if torch.is_tensor(val) else [x.to(DEV) for x in val])
+           for key, val in cpu.items()}
+    out, lse, idx, sc, outs = run_stages(inp, w, row_chunk=max(1, Lq // 3))
+    rows = rows_for(B, Lq, range(Lq))
+    oracle_check_rows(inp, w, rows, out, lse, idx, sc, outs)
+
+
+# ------------------------------------------------- full-size, sampled rows
+
+FULL = ["prefill8k", "prefill32k", "moe64k"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_prefill_sampled_rows(name):
+    w = gen.WORKLOADS[name]
+    inp = gen.make_inputs(w, seed=0, device=DEV)
+    chunk = 4096 if w.Lq > 8192 else w.Lq
+    out, lse, idx, outs_list = hs.block(inp["q"], inp["k"], inp["v"], inp["q_sparse"], inp["gate"],
+                                        w.topk, w.window, row_chunk=chunk)[0:4]
+    sp = [hs.sparse_attn(qs, inp["k"], inp["v"], idx, gt, w.window, want_branches=True)
+          for qs, gt in zip(inp["q_sparse"], inp["gate"])]
+    torch.cuda.synchronize()
+    for n in range(w.n_sparse):
+        assert torch.equal(sp[n][0], outs_list[n])
+    n_rand = {"prefill8k": 96, "prefill32k": 48, "moe64k": 24}[name]
+    rows = rows_for(w.B, w.Lq, gen.sample_rows(w.Lq, w.topk, w.window, n_random=n_rand, seed=0,
+                                               edge=8))
+    oracle_check_rows(inp, w, rows, out, lse, idx, None, sp)
+
+
+def test_full_size_decode_sampled_batches():
+    w = gen.WORKLOADS["decode"]
+    inp = gen.make_inputs(w, seed=0, device=DEV)
+    out, lse, idx, outs_list = hs.block(inp["q"], inp["k"], inp["v"], inp["q_sparse"], inp["gate"],
+                                        w.topk, w.window)
+    sp = [hs.sparse_attn(qs, inp["k"], inp["v"], idx, gt, w.window, want_branches=True)
+          for qs, gt in zip(inp["q_sparse"], inp["gate"])]
+    torch.cuda.synchronize()
+    for b in (0, 21, 42, 63):
+        one = {"q": inp["q"][b:b + 1], "k": inp["k"][b:b + 1], "v": inp["v"][b:b + 1],
+               "q_sparse": [x[b:b + 1] for x in inp["q_sparse"]],
+               "gate": [x[b:b + 1] for x in inp["gate"]]}
+        w1 = w.with_(B=1)
+        oracle_check_rows(one, w1, [(0, 0)], out[b:b + 1], lse[b:b + 1], idx[b:b + 1], None,
+                          [tuple(t[b:b + 1] for t in s) for s in sp])
