@@ -493,10 +493,14 @@ def main():
     ap.add_argument("--row-chunk", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    ap.add_argument("--seq", type=int, default=0,
+                    help="override the cache length (and the prefill length) for small profiling runs")
     args = ap.parse_args()
 
     from hybrid_sparse_attention_tcgen05_b200 import inputs as gen
     w = gen.WORKLOADS[args.workload]
+    if args.seq > 0:
+        w = w.with_(Lkv=args.seq, Lq=1 if w.Lq == 1 else args.seq, name=f"{w.name}@{args.seq}")
     world, rank, local = dist_env()
 
     if args.impl == "reference":
