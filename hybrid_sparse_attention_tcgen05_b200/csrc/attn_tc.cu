@@ -1,0 +1,616 @@
+// Tensor-core (tcgen05 / TMEM / TMA) kernels for the full layer of the
+// hybrid block, bf16 inputs, head dim 128:
+//
+//   attn_fwd_tc    : O and LSE (and per-row softmax statistics) of causal GQA
+//                    attention, flash-style online softmax over 128-key tiles.
+//   attn_scores_tc : the importance scores, a second pass over the keys that
+//                    re-computes q.k on the tensor cores and turns it into
+//                    exact probabilities with the saved statistics, summed
+//                    over the query heads that share a KV head.
+//
+// Method: HySparse abstract (the full attention layer is the oracle that
+// picks the tokens each following sparse layer attends to); the
+// intelliparadigm write-up, section 2.1 (full layer as the hub that computes
+// token importance) and section 3.1 (index sharing).  The tiling is the IO-
+// aware exact attention the ultralytics glossary names (FlashAttention):
+// online softmax, log-sum-exp saved for reuse.
+//
+// Forward kernel layout (one CTA = 128 query rows x 2 query heads of one KV
+// group, so each K/V tile is loaded once for two Q tiles):
+//   warps 0-3  softmax for Q tile 0 (thread t owns row t = TMEM lane t)
+//   warps 4-7  softmax for Q tile 1
+//   warp 8     TMA producer (Q tiles once, then K_j, V_j through a 4-slot ring)
+//   warp 9     MMA issuer (one thread)
+// TMEM (512 columns): S0 | S1 | O0 | O1, 128 f32 columns each.  P (bf16) is
+// written over the first 64 columns of its S tile and fed to the PV MMA
+// straight from TMEM.  MMAs issued by one thread execute in order, so
+// S_{j+1} = Q K_{j+1}^T may be issued right after O += P_j V_j.
+// The running max is only moved when it grows by more than 8 (log2 units);
+// the final normalisation uses the same reference, so the result is exact.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_util.cuh"
+
+namespace hs {
+namespace tc {
+namespace {
+
+constexpr int BM = 128;                 // query rows per tile
+constexpr int BN = 128;                 // keys per tile
+constexpr int HD = 128;                 // head dim
+constexpr int TILE = BM * HD * 2;       // one 128x128 bf16 tile: 32 KB
+constexpr int HALF = TILE / 2;          // one 64-column swizzled half: 16 KB
+constexpr int KV_STAGES = 4;
+constexpr int FWD_THREADS = 320;
+constexpr uint64_t kDrainNs = 1000000000ull;
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Wait that ignores the abort flag: used only to drain our own in-flight
+// copies / MMAs before the CTA exits.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+    int dummy = 0;
+    mbar_wait(bar, parity, kDrainNs, &dummy);
+}
+
+// S = Q K^T for one 128x128 tile: 8 MMAs of K=16 along the head dim.  Both
+// operands are K-major 128-byte-swizzled [128][64] halves 16 KB apart.
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
+    constexpr uint32_t I = idesc_bf16(128, 128, false, false);
+#pragma unroll
+    for (int kk = 0; kk < HD / 16; ++kk) {
+        const uint32_t o = (kk >> 2) * HALF + (kk & 3) * 32;
+        mma_ss(d_tmem, sdesc_sw128(q_addr + o, 16, 1024), sdesc_sw128(k_addr + o, 16, 1024), I,
+               kk > 0 ? 1u : 0u);
+    }
+}
+
+// O (+)= P V: P is 128x128 bf16 in TMEM (64 columns), V a [128 keys][128 d]
+// tile stored as two [128][64] swizzled halves -> N(=d)-major B operand.
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr,
+                                         bool accumulate) {
+    constexpr uint32_t I = idesc_bf16(128, 128, false, true);
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; ++kk) {
+        mma_ts(d_tmem, p_tmem + kk * 8, sdesc_sw128(v_addr + kk * 2048, HALF, 1024), I,
+               (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+struct FwdBars {
+    uint64_t q_full;
+    uint64_t kv_full[KV_STAGES];
+    uint64_t kv_empty[KV_STAGES];
+    uint64_t s_full[2];
+    uint64_t p_full[2];
+    uint64_t o_final[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+constexpr size_t kFwdSmem = 1024 + 2 * TILE + KV_STAGES * TILE + sizeof(FwdBars);
+
+struct FwdParams {
+    int Lq, Lkv, Hq, Hkv, G;
+    int row_begin, row_end;
+    float scale_log2;
+    __nv_bfloat16 *out;
+    float *lse;
+    float2 *stats;
+    unsigned int *status;
+    unsigned long long wait_ns;
+};
+
+__global__ void __launch_bounds__(FWD_THREADS, 1)
+attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+            const __grid_constant__ CUtensorMap tv, const FwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    uint8_t *sq = smem;
+    uint8_t *skv = smem + 2 * TILE;
+    FwdBars *bars = reinterpret_cast<FwdBars *>(smem + 2 * TILE + KV_STAGES * TILE);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tile = gridDim.x - 1 - blockIdx.x;  // heaviest row tiles first
+    const int r0 = p.row_begin + tile * BM;
+    const int r_end = min(r0 + BM, p.row_end);
+    const int h0 = 2 * blockIdx.y;
+    const int g = h0 / p.G;
+    const int b = blockIdx.z;
+    const int off = p.Lkv - p.Lq;
+    const int pos_first = off + r0;
+    const int pos_last = off + r_end - 1;
+    const int n_kv = pos_last / BN + 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bars->q_full), 1);
+        for (int s = 0; s < KV_STAGES; ++s) {
+            mbar_init(smem_u32(&bars->kv_full[s]), 1);
+            mbar_init(smem_u32(&bars->kv_empty[s]), 1);
+        }
+        for (int w = 0; w < 2; ++w) {
+            mbar_init(smem_u32(&bars->s_full[w]), 1);
+            mbar_init(smem_u32(&bars->p_full[w]), 128);
+            mbar_init(smem_u32(&bars->o_final[w]), 1);
+        }
+        mbar_init(smem_u32(&bars->drain), 1);
+        bars->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&bars->tmem_base), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    volatile int *abort = &bars->abort;
+
+    if (warp == 8) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch(&tq);
+            tma_prefetch(&tk);
+            tma_prefetch(&tv);
+            const uint32_t qb = smem_u32(&bars->q_full);
+            mbar_expect_tx(qb, 2 * TILE);
+            for (int s = 0; s < 2; ++s)
+                for (int hf = 0; hf < 2; ++hf)
+                    tma_load_4d(smem_u32(sq + s * TILE + hf * HALF), &tq, qb, hf * 64, h0 + s, r0, b);
+            int issued = 0;
+            for (int it = 0; it < 2 * n_kv; ++it) {
+                const int slot = it % KV_STAGES, use = it / KV_STAGES;
+                if (!mbar_wait(smem_u32(&bars->kv_empty[slot]), (use & 1) ^ 1, p.wait_ns, abort)) break;
+                const uint32_t fb = smem_u32(&bars->kv_full[slot]);
+                mbar_expect_tx(fb, TILE);
+                const CUtensorMap *m = (it & 1) ? &tv : &tk;
+                const int j = it >> 1;
+                for (int hf = 0; hf < 2; ++hf)
+                    tma_load_4d(smem_u32(skv + slot * TILE + hf * HALF), m, fb, hf * 64, g, j * BN, b);
+                issued = it + 1;
+            }
+            if (*abort) {  // let our own copies land before the CTA goes away
+                mbar_drain(qb, 0);
+                for (int it = issued > KV_STAGES ? issued - KV_STAGES : 0; it < issued; ++it)
+                    mbar_drain(smem_u32(&bars->kv_full[it % KV_STAGES]), (it / KV_STAGES) & 1);
+            }
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
+            const uint32_t q0 = smem_u32(sq), q1 = smem_u32(sq + TILE);
+            bool ok = mbar_wait(smem_u32(&bars->q_full), 0, p.wait_ns, abort);
+            // S for tile 0
+            if (ok) ok = mbar_wait(smem_u32(&bars->kv_full[0]), 0, p.wait_ns, abort);
+            if (ok) {
+                tc_fence_after();
+                const uint32_t ka = smem_u32(skv);
+                issue_qk(tS0, q0, ka);
+                mma_commit(smem_u32(&bars->s_full[0]));
+                issue_qk(tS1, q1, ka);
+                mma_commit(smem_u32(&bars->s_full[1]));
+                mma_commit(smem_u32(&bars->kv_empty[0]));
+            }
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int itV = 2 * j + 1, slotV = itV % KV_STAGES;
+                const int itK = 2 * j + 2, slotK = itK % KV_STAGES;
+                const bool has_next = j + 1 < n_kv;
+                const uint32_t va = smem_u32(skv + slotV * TILE);
+                const uint32_t ka = smem_u32(skv + slotK * TILE);
+                if (!(ok = mbar_wait(smem_u32(&bars->kv_full[slotV]), (itV / KV_STAGES) & 1, p.wait_ns, abort))) break;
+                if (!(ok = mbar_wait(smem_u32(&bars->p_full[0]), j & 1, p.wait_ns, abort))) break;
+                tc_fence_after();
+                issue_pv(tO0, tS0, va, j > 0);
+                if (!has_next) mma_commit(smem_u32(&bars->o_final[0]));
+                if (has_next) {
+                    if (!(ok = mbar_wait(smem_u32(&bars->kv_full[slotK]), (itK / KV_STAGES) & 1, p.wait_ns, abort))) break;
+                    tc_fence_after();
+                    issue_qk(tS0, q0, ka);
+                    mma_commit(smem_u32(&bars->s_full[0]));
+                }
+                if (!(ok = mbar_wait(smem_u32(&bars->p_full[1]), j & 1, p.wait_ns, abort))) break;
+                tc_fence_after();
+                issue_pv(tO1, tS1, va, j > 0);
+                mma_commit(smem_u32(&bars->kv_empty[slotV]));
+                if (!has_next) mma_commit(smem_u32(&bars->o_final[1]));
+                if (has_next) {
+                    issue_qk(tS1, q1, ka);
+                    mma_commit(smem_u32(&bars->s_full[1]));
+                    mma_commit(smem_u32(&bars->kv_empty[slotK]));
+                }
+            }
+            // all MMAs this thread issued have completed before TMEM is freed
+            mma_commit(smem_u32(&bars->drain));
+            mbar_drain(smem_u32(&bars->drain), 0);
+        }
+    } else {
+        // ------------------------------------------------ softmax warpgroups
+        const int w = warp >> 2;
+        const int tw = threadIdx.x - 128 * w;
+        const int row = r0 + tw;
+        const bool valid = row < r_end;
+        const int pos = off + min(row, r_end - 1);
+        const uint32_t lane_off = (uint32_t)(tw & ~31) << 16;
+        const uint32_t tS = tmem + lane_off + (uint32_t)(w * 128);
+        const uint32_t tO = tmem + lane_off + 256u + (uint32_t)(w * 128);
+        const float c2 = p.scale_log2;
+        float m = -INFINITY, l = 0.f, lc = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[w]), j & 1, p.wait_ns, abort));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t r[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
+            tmem_wait_ld();
+            float s[128];
+#pragma unroll
+            for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(r[c >> 5][c & 31]);
+            if (j * BN + BN - 1 > pos_first) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (j * BN + c > pos) s[c] = -INFINITY;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+            const float mx2 = mx * c2;
+            if (__any_sync(0xffffffffu, mx2 > m + 8.0f)) {
+                const float m_new = fmaxf(m, mx2);
+                if (j > 0) {
+                    const float corr = ex2(m - m_new);
+                    l *= corr;
+                    lc *= corr;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + 32 * c, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+                        tmem_st32(tO + 32 * c, o);
+                    }
+                    tmem_wait_st();
+                }
+                m = m_new;
+            }
+            float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int c = hf * 64 + 2 * e;
+                    const float a = ex2(fmaf(s[c], c2, -m));
+                    const float bb = ex2(fmaf(s[c + 1], c2, -m));
+                    if (e & 1) { ps2 += a; ps3 += bb; } else { ps0 += a; ps1 += bb; }
+                    pk[e] = pack_bf16(a, bb);
+                }
+                tmem_st32(tS + 32 * hf, pk);
+            }
+            tmem_wait_st();
+            const float ts = (ps0 + ps1) + (ps2 + ps3);
+            const float y = ts - lc;
+            const float t = l + y;
+            lc = (t - l) - y;
+            l = t;
+            tc_fence_before();
+            mbar_arrive(smem_u32(&bars->p_full[w]));
+        }
+        const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(smem_u32(&bars->o_final[w]), 0, p.wait_ns, abort));
+        if (fin) {
+            tc_fence_after();
+            const int h = h0 + w;
+            const float inv_l = 1.0f / l;
+            __nv_bfloat16 *orow = p.out + (((size_t)b * p.Lq + row) * p.Hq + h) * HD;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + 32 * c, o);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+                if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
+            }
+            if (valid) {
+                const size_t si = ((size_t)b * p.Hq + h) * p.Lq + row;
+                p.lse[si] = (m + log2f(l)) * kLn2;
+                if (p.stats) p.stats[si] = make_float2(m, inv_l);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+    if (threadIdx.x == 0 && bars->abort) report(p.status, HS_ERR_TIMEOUT);
+}
+
+// ------------------------------------------------------------------ scores
+
+constexpr int SC_Q_STAGES = 3;
+constexpr int SC_K_STAGES = 2;
+constexpr int SC_BUFS = 4;
+constexpr int SC_THREADS = 192;   // warps 0-3 scores, 4 TMA, 5 MMA
+
+struct ScBars {
+    uint64_t q_full[SC_Q_STAGES], q_empty[SC_Q_STAGES];
+    uint64_t k_full[SC_K_STAGES], k_empty[SC_K_STAGES];
+    uint64_t s_full[SC_BUFS], s_free[SC_BUFS];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+constexpr size_t kScSmem = 1024 + (SC_Q_STAGES + SC_K_STAGES) * TILE + sizeof(ScBars);
+
+struct ScParams {
+    int Lq, Lkv, Hq, Hkv, G;
+    int row_begin, row_end, row_count;
+    float scale_log2;
+    const float2 *stats;
+    float *scores;
+    long long ld;
+    unsigned int *status;
+    unsigned long long wait_ns;
+};
+
+__global__ void __launch_bounds__(SC_THREADS, 1)
+attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+               const ScParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    uint8_t *sq = smem;
+    uint8_t *sk = smem + SC_Q_STAGES * TILE;
+    ScBars *bars = reinterpret_cast<ScBars *>(smem + (SC_Q_STAGES + SC_K_STAGES) * TILE);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tile = gridDim.x - 1 - blockIdx.x;
+    const int r0 = p.row_begin + tile * BM;
+    const int r_end = min(r0 + BM, p.row_end);
+    const int g = blockIdx.y;
+    const int b = blockIdx.z;
+    const int G = p.G;
+    const int off = p.Lkv - p.Lq;
+    const int pos_last = off + r_end - 1;
+    const int n_kv = pos_last / BN + 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < SC_Q_STAGES; ++s) {
+            mbar_init(smem_u32(&bars->q_full[s]), 1);
+            mbar_init(smem_u32(&bars->q_empty[s]), 1);
+        }
+        for (int s = 0; s < SC_K_STAGES; ++s) {
+            mbar_init(smem_u32(&bars->k_full[s]), 1);
+            mbar_init(smem_u32(&bars->k_empty[s]), 1);
+        }
+        for (int s = 0; s < SC_BUFS; ++s) {
+            mbar_init(smem_u32(&bars->s_full[s]), 1);
+            mbar_init(smem_u32(&bars->s_free[s]), 128);
+        }
+        mbar_init(smem_u32(&bars->drain), 1);
+        bars->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&bars->tmem_base), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    volatile int *abort = &bars->abort;
+
+    if (warp == 4) {
+        if (lane == 0) {
+            tma_prefetch(&tq);
+            tma_prefetch(&tk);
+            int k_issued = 0, q_issued = 0;
+            bool ok = true;
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int sk_ = j % SC_K_STAGES;
+                if (!(ok = mbar_wait(smem_u32(&bars->k_empty[sk_]), ((j / SC_K_STAGES) & 1) ^ 1, p.wait_ns, abort))) break;
+                const uint32_t kb = smem_u32(&bars->k_full[sk_]);
+                mbar_expect_tx(kb, TILE);
+                for (int hf = 0; hf < 2; ++hf)
+                    tma_load_4d(smem_u32(sk + sk_ * TILE + hf * HALF), &tk, kb, hf * 64, g, j * BN, b);
+                k_issued = j + 1;
+                for (int hh = 0; hh < G; ++hh) {
+                    const int it = j * G + hh, sq_ = it % SC_Q_STAGES;
+                    if (!(ok = mbar_wait(smem_u32(&bars->q_empty[sq_]), ((it / SC_Q_STAGES) & 1) ^ 1, p.wait_ns, abort))) break;
+                    const uint32_t qb = smem_u32(&bars->q_full[sq_]);
+                    mbar_expect_tx(qb, TILE);
+                    for (int hf = 0; hf < 2; ++hf)
+                        tma_load_4d(smem_u32(sq + sq_ * TILE + hf * HALF), &tq, qb, hf * 64, g * G + hh, r0, b);
+                    q_issued = it + 1;
+                }
+            }
+            if (*abort) {
+                for (int j = k_issued > SC_K_STAGES ? k_issued - SC_K_STAGES : 0; j < k_issued; ++j)
+                    mbar_drain(smem_u32(&bars->k_full[j % SC_K_STAGES]), (j / SC_K_STAGES) & 1);
+                for (int it = q_issued > SC_Q_STAGES ? q_issued - SC_Q_STAGES : 0; it < q_issued; ++it)
+                    mbar_drain(smem_u32(&bars->q_full[it % SC_Q_STAGES]), (it / SC_Q_STAGES) & 1);
+            }
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            bool ok = true;
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int sk_ = j % SC_K_STAGES;
+                if (!(ok = mbar_wait(smem_u32(&bars->k_full[sk_]), (j / SC_K_STAGES) & 1, p.wait_ns, abort))) break;
+                const uint32_t ka = smem_u32(sk + sk_ * TILE);
+                for (int hh = 0; hh < G; ++hh) {
+                    const int it = j * G + hh, sq_ = it % SC_Q_STAGES, buf = it % SC_BUFS;
+                    if (!(ok = mbar_wait(smem_u32(&bars->q_full[sq_]), (it / SC_Q_STAGES) & 1, p.wait_ns, abort))) break;
+                    if (!(ok = mbar_wait(smem_u32(&bars->s_free[buf]), ((it / SC_BUFS) & 1) ^ 1, p.wait_ns, abort))) break;
+                    tc_fence_after();
+                    issue_qk(tmem + (uint32_t)(buf * 128), smem_u32(sq + sq_ * TILE), ka);
+                    mma_commit(smem_u32(&bars->s_full[buf]));
+                    mma_commit(smem_u32(&bars->q_empty[sq_]));
+                }
+                if (ok) mma_commit(smem_u32(&bars->k_empty[sk_]));
+            }
+            mma_commit(smem_u32(&bars->drain));
+            mbar_drain(smem_u32(&bars->drain), 0);
+        }
+    } else {
+        // ------------------------------------------------ score warps
+        const int tw = threadIdx.x;
+        const int row = r0 + tw;
+        const bool valid = row < r_end;
+        const int pos = off + min(row, r_end - 1);
+        const uint32_t lane_off = (uint32_t)(tw & ~31) << 16;
+        const float c2 = p.scale_log2;
+        float *srow = valid ? p.scores + (((size_t)b * p.Hkv + g) * p.row_count + (row - p.row_begin)) * p.ld
+                            : nullptr;
+        const bool vec4 = (p.ld & 3) == 0;
+        bool ok = true;
+        for (int j = 0; ok && j < n_kv; ++j) {
+            float acc[128];
+#pragma unroll
+            for (int c = 0; c < 128; ++c) acc[c] = 0.f;
+            for (int hh = 0; hh < G; ++hh) {
+                const int it = j * G + hh, buf = it % SC_BUFS;
+                const float2 st = valid ? p.stats[((size_t)b * p.Hq + g * G + hh) * p.Lq + row]
+                                        : make_float2(0.f, 0.f);
+                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[buf]), (it / SC_BUFS) & 1, p.wait_ns, abort));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t tS = tmem + lane_off + (uint32_t)(buf * 128);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tS + 32 * c, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        acc[32 * c + e] = fmaf(ex2(fmaf(__uint_as_float(r[e]), c2, -st.x)), st.y, acc[32 * c + e]);
+                }
+                tc_fence_before();
+                mbar_arrive(smem_u32(&bars->s_free[buf]));
+            }
+            if (!ok) break;
+            if (valid) {
+                const int j0 = j * BN;
+                const int lim = min(BN, p.Lkv - j0);      // columns inside the cache
+                const int keep = min(lim, pos - j0 + 1);  // causal columns
+                float *dst = srow + j0;
+                if (vec4 && lim == BN) {
+#pragma unroll
+                    for (int c = 0; c < 128; c += 4) {
+                        float4 v4 = make_float4(c < keep ? acc[c] : 0.f, c + 1 < keep ? acc[c + 1] : 0.f,
+                                                c + 2 < keep ? acc[c + 2] : 0.f, c + 3 < keep ? acc[c + 3] : 0.f);
+                        *reinterpret_cast<float4 *>(dst + c) = v4;
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (c < lim) dst[c] = c < keep ? acc[c] : 0.f;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+    if (threadIdx.x == 0 && bars->abort) report(p.status, HS_ERR_TIMEOUT);
+}
+
+// ----------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// [B][L][H][128] bf16 -> 4-D map (d, H, L, B) with a {64, 1, 128, 1} box,
+// 128-byte swizzle; rows past L read as zeros.
+bool make_map(CUtensorMap *m, const void *base, int H, int L, int B) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)HD * 2, (cuuint64_t)HD * 2 * H, (cuuint64_t)HD * 2 * H * L};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)BM, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+}  // namespace tc
+
+bool full_attn_tc_supported(const Shape &s) {
+    return s.dtype == HS_BF16 && s.d == 128 && (s.G() % 2) == 0 && s.Lkv < (1 << 24);
+}
+
+cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void *k, const void *v,
+                                       void *out, float *lse, float *scores, long long ld,
+                                       int row_begin, int row_count, float2 *stats,
+                                       unsigned int *status, unsigned long long wait_ns,
+                                       cudaStream_t st) {
+    using namespace tc;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, s.Hq, s.Lq, s.B) || !make_map(&mk, k, s.Hkv, s.Lkv, s.B) ||
+        !make_map(&mv, v, s.Hkv, s.Lkv, s.B))
+        return cudaErrorInvalidValue;
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdSmem);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(attn_scores_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScSmem);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    const int n_tiles = (row_count + BM - 1) / BM;
+    FwdParams fp{s.Lq, s.Lkv, s.Hq, s.Hkv, s.G(), row_begin, row_begin + row_count,
+                 s.scale * kLog2e, (__nv_bfloat16 *)out, lse, stats, status, wait_ns};
+    attn_fwd_tc<<<dim3(n_tiles, s.Hq / 2, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || scores == nullptr) return e;
+    ScParams sp{s.Lq, s.Lkv, s.Hq, s.Hkv, s.G(), row_begin, row_begin + row_count, row_count,
+                s.scale * kLog2e, stats, scores, ld, status, wait_ns};
+    attn_scores_tc<<<dim3(n_tiles, s.Hkv, s.B), SC_THREADS, kScSmem, st>>>(mq, mk, sp);
+    return cudaGetLastError();
+}
+
+}  // namespace hs

@@ -3,6 +3,7 @@
 // the contract of every call.
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "common.cuh"
@@ -16,6 +17,10 @@ constexpr int kMaxTopk = 4096;
 constexpr int kMaxWindow = 1024;
 constexpr int kMaxGroup = 32;
 constexpr int kMaxLen = 1 << 24;
+
+// Query rows below which the tensor-core full layer is not used (a 128-row
+// tile would be mostly empty; decode takes the CUDA-core path).
+constexpr int kTcMinRows = 64;
 
 bool aligned16(const void *p) { return p != nullptr && ((uintptr_t)p & 15u) == 0; }
 
@@ -72,7 +77,13 @@ int check_full_args(const Shape &s, const void *q, const void *k, const void *v,
 
 int run_full(const Shape &s, const void *q, const void *k, const void *v, void *out, float *lse,
              float *scores, long long ld, int row_begin, int row_count, void *ws, cudaStream_t st) {
-    (void)ws;
+    if (full_attn_tc_supported(s) && s.Lq >= kTcMinRows) {
+        char *w = reinterpret_cast<char *>(ws);
+        float2 *stats = reinterpret_cast<float2 *>(w + ws_layout(s, 1, row_count).stats);
+        unsigned int *status = reinterpret_cast<unsigned int *>(ws);
+        return cuda_status(full_attn_scores_tc_launch(s, q, k, v, out, lse, scores, ld, row_begin,
+                                                      row_count, stats, status, wait_limit_ns(), st));
+    }
     return cuda_status(full_attn_scores_simt_launch(s, q, k, v, out, lse, scores, ld, row_begin,
                                                     row_count, st));
 }
@@ -91,6 +102,15 @@ int run_sparse(const Shape &s, const void *q, const void *k, const void *v, cons
 }
 
 }  // namespace
+
+unsigned long long wait_limit_ns() {
+    // HYSPARSE_WAIT_LIMIT_NS lowers the bound on in-kernel waits; the tests
+    // set it to 0 to drive the timeout path without hanging anything.
+    const char *e = getenv("HYSPARSE_WAIT_LIMIT_NS");
+    if (e && *e) return strtoull(e, nullptr, 10);
+    return 1000000000ull;
+}
+
 }  // namespace hs
 
 using namespace hs;

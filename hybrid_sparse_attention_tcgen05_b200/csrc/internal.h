@@ -27,6 +27,18 @@ cudaError_t sparse_attn_simt_launch(const Shape &s, const void *q, const void *k
                                     void *out, void *og, void *ol, unsigned int *status,
                                     cudaStream_t st);
 
+// attn_tc.cu (bf16, d = 128, even group size)
+bool full_attn_tc_supported(const Shape &s);
+cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void *k, const void *v,
+                                       void *out, float *lse, float *scores, long long ld,
+                                       int row_begin, int row_count, float2 *stats,
+                                       unsigned int *status, unsigned long long wait_ns,
+                                       cudaStream_t st);
+
+// Upper bound (ns) on any single barrier wait inside a kernel; after it the
+// kernel records HS_ERR_TIMEOUT in the workspace status word and returns.
+unsigned long long wait_limit_ns();
+
 // topk.cu
 cudaError_t topk_launch(const Shape &s, const float *scores, long long ld, int row_begin,
                         int row_count, int topk, int32_t *idx, cudaStream_t st);
