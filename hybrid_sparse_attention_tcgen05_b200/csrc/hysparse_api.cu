@@ -97,6 +97,9 @@ int run_sparse(const Shape &s, const void *q, const void *k, const void *v, cons
                int topk, const float *gate, int window, void *out, void *og, void *ol, void *ws,
                cudaStream_t st) {
     unsigned int *status = reinterpret_cast<unsigned int *>(ws);
+    if (sparse_mma_supported(s))
+        return cuda_status(sparse_attn_mma_launch(s, q, k, v, idx, topk, gate, window, out, og, ol, status,
+                                                  wait_limit_ns(), st));
     return cuda_status(sparse_attn_simt_launch(s, q, k, v, idx, topk, gate, window, out, og, ol,
                                                status, st));
 }

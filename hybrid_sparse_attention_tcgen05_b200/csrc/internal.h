@@ -35,6 +35,13 @@ cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void
                                        unsigned int *status, unsigned long long wait_ns,
                                        cudaStream_t st);
 
+// sparse_mma.cu (bf16, d = 128, G <= 16)
+bool sparse_mma_supported(const Shape &s);
+cudaError_t sparse_attn_mma_launch(const Shape &s, const void *q, const void *k, const void *v,
+                                   const int32_t *idx, int topk, const float *gate, int window, void *out,
+                                   void *og, void *ol, unsigned int *status, unsigned long long wait_ns,
+                                   cudaStream_t st);
+
 // Upper bound (ns) on any single barrier wait inside a kernel; after it the
 // kernel records HS_ERR_TIMEOUT in the workspace status word and returns.
 unsigned long long wait_limit_ns();

@@ -1,0 +1,394 @@
+// Sparse layer of the hybrid block on the tensor cores (bf16, d = 128):
+// global branch over each row's top-k key set + causal 128-token window
+// branch + sigmoid gate, reading the full layer's KV cache and writing no KV.
+//
+// Method: intelliparadigm write-up section 2.2 (dual-branch sparse attention:
+// a global branch over the TopK indices of the preceding full layer, a local
+// 128-token sliding window, out = gate*global + (1-gate)*local with a sigmoid
+// gate) and section 3.1 (the sparse layers only read the full layer's cache).
+//
+// One warp owns one (batch, query row, KV head) item: the G query heads of
+// that group share the item's key list.  Keys are gathered 32 at a time:
+// each lane issues one 256-byte bulk copy for its key's K row and one for its
+// V row into a 3-stage shared-memory ring (rows padded to 272 bytes so
+// ldmatrix is conflict-free); completion is counted in bytes on a per-stage
+// mbarrier.  The maths runs on mma.sync m16n8k16 with the keys as M (so a
+// small group of heads only pads N to 8 or 16): S^T = K Q^T, an online
+// softmax per head column, then O^T += V^T P^T where movmatrix turns the
+// S^T accumulator fragment into the B operand.  The window branch reuses the
+// same pipeline over the contiguous key range; both branches are merged by
+// the gate in registers and the G output rows are written once.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_util.cuh"
+
+namespace hs {
+namespace tc {
+namespace {
+
+constexpr int SW = 4;             // warps (items) per CTA
+constexpr int CH = 32;            // keys per chunk (one per lane)
+constexpr int ST = 3;             // pipeline stages per warp
+constexpr int RS = 272;           // padded row stride in shared memory (bytes)
+constexpr int STAGE_BYTES = 2 * CH * RS;
+
+template <int NB>
+struct SpSmem {
+    static constexpr int QB = 8 * NB * RS;               // Q staging / output staging
+    static constexpr int WARP_BYTES = ST * STAGE_BYTES + QB;
+    static constexpr size_t bytes = (size_t)SW * WARP_BYTES;
+};
+
+__device__ __forceinline__ float ex2f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Online softmax + PV state of one branch for NB blocks of 8 heads.
+template <int NB>
+struct Branch {
+    float m[NB][2], l[NB][2], o[NB][8][4];
+    __device__ void init() {
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) { m[nb][e] = -INFINITY; l[nb][e] = 0.f; }
+#pragma unroll
+            for (int md = 0; md < 8; ++md)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) o[nb][md][r] = 0.f;
+        }
+    }
+};
+
+struct SpParams {
+    const __nv_bfloat16 *q, *k, *v;
+    const int32_t *idx;
+    const float *gate;
+    __nv_bfloat16 *out, *out_g, *out_l;
+    int B, Lq, Lkv, Hq, Hkv, G, topk, window;
+    float scale_log2;
+    unsigned int *status;
+    unsigned long long wait_ns;
+};
+
+template <int NB>
+__device__ __forceinline__ void issue_chunk(const SpParams &p, const int32_t *list, bool from_list, int lo,
+                                            int n_list, int t0, int pos, const __nv_bfloat16 *kb,
+                                            const __nv_bfloat16 *vb, uint8_t *stage, uint32_t bar,
+                                            uint32_t &vmask, int lane) {
+    const int t = t0 + lane;
+    int key = -1;
+    if (t < n_list) {
+        key = from_list ? __ldg(list + t) : lo + t;
+        if (key < -1 || key > pos) {
+            report(p.status, HS_ERR_INVALID_INDEX);
+            key = -1;
+        }
+    }
+    const bool valid = key >= 0;
+    vmask = __ballot_sync(0xffffffffu, valid);
+    if (lane == 0) mbar_expect_tx(bar, (uint32_t)__popc(vmask) * 512u);
+    __syncwarp();
+    uint8_t *krow = stage + lane * RS;
+    uint8_t *vrow = stage + CH * RS + lane * RS;
+    if (valid) {
+        const size_t ro = (size_t)key * p.Hkv * 128;
+        bulk_g2s(smem_u32(krow), kb + ro, 256, bar);
+        bulk_g2s(smem_u32(vrow), vb + ro, 256, bar);
+    } else {
+        const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            reinterpret_cast<uint4 *>(krow)[c] = z;
+            reinterpret_cast<uint4 *>(vrow)[c] = z;
+        }
+    }
+}
+
+template <int NB>
+__device__ __forceinline__ void compute_chunk(const uint8_t *stage, uint32_t vmask, const uint32_t (&bq)[NB][8][2],
+                                              float c2, Branch<NB> &br, int lane) {
+    const uint32_t ks_base = smem_u32(stage);
+    const uint32_t vs_base = smem_u32(stage + CH * RS);
+    float c[NB][2][4];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) c[nb][mt][r] = 0.f;
+    // S^T[32 keys x 8NB heads] = K Q^T
+    const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;
+    const int acol = (lane >> 4) * 8;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(ks_base + (16 * mt + arow) * RS + (16 * ks + acol) * 2, a0, a1, a2, a3);
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) mma16816(c[nb][mt], a0, a1, a2, a3, bq[nb][ks][0], bq[nb][ks][1]);
+        }
+    }
+    // online softmax per head column (keys spread over lane/4 and the two row halves)
+    bool kv[2][2];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh) kv[mt][rh] = (vmask >> (16 * mt + (lane >> 2) + 8 * rh)) & 1u;
+    uint32_t bp[NB][2][2];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            float x[2][2];
+            float cm = -INFINITY;
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int rh = 0; rh < 2; ++rh) {
+                    x[mt][rh] = kv[mt][rh] ? c[nb][mt][2 * rh + e] * c2 : -INFINITY;
+                    cm = fmaxf(cm, x[mt][rh]);
+                }
+            cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 4));
+            cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 8));
+            cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 16));
+            const float mn = fmaxf(br.m[nb][e], cm);
+            const float corr = (mn == -INFINITY) ? 1.f : ex2f(br.m[nb][e] - mn);
+            float ps = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int rh = 0; rh < 2; ++rh) {
+                    const float pv = (mn == -INFINITY) ? 0.f : ex2f(x[mt][rh] - mn);
+                    c[nb][mt][2 * rh + e] = pv;
+                    ps += pv;
+                }
+            ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 16);
+            br.l[nb][e] = br.l[nb][e] * corr + ps;
+            br.m[nb][e] = mn;
+#pragma unroll
+            for (int md = 0; md < 8; ++md) {
+                br.o[nb][md][e] *= corr;
+                br.o[nb][md][2 + e] *= corr;
+            }
+        }
+        // P^T fragments (keys x heads) -> B operand (k = keys, n = heads)
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            bp[nb][mt][0] = movm_t(pack_bf16(c[nb][mt][0], c[nb][mt][1]));
+            bp[nb][mt][1] = movm_t(pack_bf16(c[nb][mt][2], c[nb][mt][3]));
+        }
+    }
+    // O^T[128 d x 8NB heads] += V^T P^T
+    const int vrow = (lane & 7) + ((lane >> 4) & 1) * 8;
+    const int vcol = ((lane >> 3) & 1) * 8;
+#pragma unroll
+    for (int md = 0; md < 8; ++md) {
+#pragma unroll
+        for (int kt = 0; kt < 2; ++kt) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(vs_base + (16 * kt + vrow) * RS + (16 * md + vcol) * 2, a0, a1, a2, a3);
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) mma16816(br.o[nb][md], a0, a1, a2, a3, bp[nb][kt][0], bp[nb][kt][1]);
+        }
+    }
+}
+
+// Everything one warp needs to run a branch's gather pipeline.
+struct WarpCtx {
+    const SpParams *p;
+    const int32_t *list;
+    const __nv_bfloat16 *kb, *vb;
+    uint8_t *wbase;
+    uint32_t bar0;
+    int lo, pos, lane;
+    float c2;
+};
+
+__device__ __forceinline__ uint32_t pick3(uint32_t s, uint32_t a, uint32_t b, uint32_t c) {
+    return s == 0 ? a : (s == 1 ? b : c);
+}
+
+// Run one branch (from_list: the top-k list, else the causal window) through
+// the ST-stage gather pipeline.  `seq` counts chunks issued by this warp so
+// far (it fixes each stage's mbarrier parity).  Returns false on abort.
+template <int NB>
+__device__ __forceinline__ bool run_branch(const WarpCtx &w, bool from_list, const uint32_t (&bq)[NB][8][2],
+                                           Branch<NB> &br, uint32_t &seq, int &aborted) {
+    static_assert(ST == 3, "pick3 assumes three stages");
+    const SpParams &p = *w.p;
+    br.init();
+    const int n_list = from_list ? p.topk : w.pos - w.lo + 1;
+    const int nch = (n_list + CH - 1) / CH;
+    const uint32_t base = seq;
+    uint32_t vm0 = 0, vm1 = 0, vm2 = 0;
+    auto issue = [&](int c) {
+        const uint32_t sq_ = base + c, s = sq_ % ST;
+        uint32_t vmask;
+        issue_chunk<NB>(p, w.list, from_list, w.lo, n_list, c * CH, w.pos, w.kb, w.vb, w.wbase + s * STAGE_BYTES,
+                        w.bar0 + 8 * s, vmask, w.lane);
+        if (s == 0) vm0 = vmask; else if (s == 1) vm1 = vmask; else vm2 = vmask;
+        seq = sq_ + 1;
+    };
+    const int pre = min(ST - 1, nch);
+    for (int c = 0; c < pre; ++c) issue(c);
+#pragma unroll 1
+    for (int c = 0; c < nch; ++c) {
+        __syncwarp();
+        if (c + ST - 1 < nch) issue(c + ST - 1);
+        const uint32_t sq_ = base + c, s = sq_ % ST;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(w.bar0 + 8 * s, (sq_ / ST) & 1, p.wait_ns, &aborted));
+        if (!ok) {
+            aborted = 1;
+            return false;
+        }
+        compute_chunk<NB>(w.wbase + s * STAGE_BYTES, pick3(s, vm0, vm1, vm2), bq, w.c2, br, w.lane);
+    }
+    return true;
+}
+
+template <int NB>
+__global__ void __launch_bounds__(SW * 32, 1) sparse_attn_mma(const SpParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ uint64_t bars[SW][ST];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long item = (long long)blockIdx.x * SW + warp;
+    if (item >= (long long)p.B * p.Lq * p.Hkv) return;   // whole warp leaves together
+    const int g = (int)(item % p.Hkv);
+    const long long bi = item / p.Hkv;
+    const int i = (int)(bi % p.Lq);
+    const int b = (int)(bi / p.Lq);
+    const int G = p.G;
+    const int pos = p.Lkv - p.Lq + i;
+    uint8_t *wbase = smem + warp * SpSmem<NB>::WARP_BYTES;
+    uint8_t *qs = wbase + ST * STAGE_BYTES;
+    const uint32_t bar0 = smem_u32(&bars[warp][0]);
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < ST; ++s) mbar_init(bar0 + 8 * s, 1);
+        fence_mbar_init();
+    }
+    // stage the group's query rows (zero rows pad the heads up to 8*NB)
+    const size_t qrow = ((size_t)b * p.Lq + i) * p.Hq + (size_t)g * G;
+    for (int e = lane; e < 8 * NB * 16; e += 32) {
+        const int h = e >> 4, cc = e & 15;
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (h < G) val = __ldg(reinterpret_cast<const uint4 *>(p.q + (qrow + h) * 128) + cc);
+        *reinterpret_cast<uint4 *>(qs + h * RS + cc * 16) = val;
+    }
+    __syncwarp();
+    uint32_t bq[NB][8][2];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int kp = 0; kp < 4; ++kp)
+            ldsm_x4(smem_u32(qs + (8 * nb + (lane & 7)) * RS + (32 * kp + 8 * (lane >> 3)) * 2),
+                    bq[nb][2 * kp][0], bq[nb][2 * kp][1], bq[nb][2 * kp + 1][0], bq[nb][2 * kp + 1][1]);
+
+    WarpCtx w;
+    w.p = &p;
+    w.kb = p.k + ((size_t)b * p.Lkv * p.Hkv + g) * 128;
+    w.vb = p.v + ((size_t)b * p.Lkv * p.Hkv + g) * 128;
+    w.list = p.idx + (((size_t)b * p.Hkv + g) * p.Lq + i) * p.topk;
+    w.wbase = wbase;
+    w.bar0 = bar0;
+    w.lo = max(0, pos - p.window + 1);
+    w.pos = pos;
+    w.lane = lane;
+    w.c2 = p.scale_log2;
+    int aborted = 0;
+    uint32_t seq = 0;
+    Branch<NB> bg, bl;
+    bool ok = run_branch<NB>(w, true, bq, bg, seq, aborted);
+    if (ok) ok = run_branch<NB>(w, false, bq, bl, seq, aborted);
+    if (!ok) {
+        // let every copy this warp issued land before the warp exits
+        for (uint32_t sq_ = seq > ST ? seq - ST : 0; sq_ < seq; ++sq_) {
+            int dummy = 0;
+            mbar_wait(bar0 + 8 * (sq_ % ST), (sq_ / ST) & 1, 1000000000ull, &dummy);
+        }
+        if (lane == 0) report(p.status, HS_ERR_TIMEOUT);
+        return;
+    }
+
+    // gate merge, stage the G output rows in shared memory, write them once
+    __syncwarp();
+    const size_t orow = qrow * 128;
+#pragma unroll 1
+    for (int which = 0; which < 3; ++which) {
+        __nv_bfloat16 *dst = which == 0 ? p.out : (which == 1 ? p.out_g : p.out_l);
+        if (dst == nullptr) continue;
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int h = 8 * nb + 2 * (lane & 3) + e;
+                const float lg = bg.l[nb][e], ll = bl.l[nb][e];
+                const float ig = lg > 0.f ? 1.f / lg : 0.f;
+                const float il = ll > 0.f ? 1.f / ll : 0.f;
+                float sg = 0.f;
+                if (h < G) {
+                    const float x = p.gate[((size_t)b * p.Lq + i) * p.Hq + (size_t)g * G + h];
+                    sg = 1.0f / (1.0f + expf(-x));
+                }
+                const float wg = which == 0 ? sg * ig : (which == 1 ? ig : 0.f);
+                const float wl = which == 0 ? (1.f - sg) * il : (which == 2 ? il : 0.f);
+#pragma unroll
+                for (int md = 0; md < 8; ++md)
+#pragma unroll
+                    for (int rh = 0; rh < 2; ++rh) {
+                        const int d = 16 * md + (lane >> 2) + 8 * rh;
+                        const float val = bg.o[nb][md][2 * rh + e] * wg + bl.o[nb][md][2 * rh + e] * wl;
+                        reinterpret_cast<__nv_bfloat16 *>(qs + h * RS)[d] = __float2bfloat16_rn(val);
+                    }
+            }
+        }
+        __syncwarp();
+        for (int e = lane; e < G * 16; e += 32) {
+            const int h = e >> 4, cc = e & 15;
+            reinterpret_cast<uint4 *>(dst + orow + (size_t)h * 128)[cc] =
+                *reinterpret_cast<const uint4 *>(qs + h * RS + cc * 16);
+        }
+        __syncwarp();
+    }
+}
+
+template <int NB>
+cudaError_t launch_nb(const SpParams &p, cudaStream_t st) {
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(sparse_attn_mma<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SpSmem<NB>::bytes);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    const long long items = (long long)p.B * p.Lq * p.Hkv;
+    const long long blocks = (items + SW - 1) / SW;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+    sparse_attn_mma<NB><<<(unsigned)blocks, SW * 32, SpSmem<NB>::bytes, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace tc
+
+bool sparse_mma_supported(const Shape &s) { return s.dtype == HS_BF16 && s.d == 128 && s.G() <= 16; }
+
+cudaError_t sparse_attn_mma_launch(const Shape &s, const void *q, const void *k, const void *v,
+                                   const int32_t *idx, int topk, const float *gate, int window, void *out,
+                                   void *og, void *ol, unsigned int *status, unsigned long long wait_ns,
+                                   cudaStream_t st) {
+    tc::SpParams p{(const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, idx, gate,
+                   (__nv_bfloat16 *)out, (__nv_bfloat16 *)og, (__nv_bfloat16 *)ol, s.B, s.Lq, s.Lkv, s.Hq,
+                   s.Hkv, s.G(), topk, window, s.scale * kLog2e, status, wait_ns};
+    return s.G() <= 8 ? tc::launch_nb<1>(p, st) : tc::launch_nb<2>(p, st);
+}
+
+}  // namespace hs
