@@ -8,11 +8,11 @@
 // gate) and section 3.1 (the sparse layers only read the full layer's cache).
 //
 // One warp owns one (batch, query row, KV head) item: the G query heads of
-// that group share the item's key list.  Keys are gathered 32 at a time:
-// each lane issues one 256-byte bulk copy for its key's K row and one for its
-// V row into a 3-stage shared-memory ring (rows padded to 272 bytes so
-// ldmatrix is conflict-free); completion is counted in bytes on a per-stage
-// mbarrier.  The maths runs on mma.sync m16n8k16 with the keys as M (so a
+// that group share the item's key list.  Keys are gathered 32 at a time with
+// cp.async 16-byte copies (each warp instruction moves two whole 256-byte K or
+// V rows, so every L2 sector fetched is used) into a 3-stage shared-memory
+// ring; rows are padded to 272 bytes so ldmatrix is conflict-free, and slots
+// of invalid keys are zero-filled by the copy itself.  The maths runs on mma.sync m16n8k16 with the keys as M (so a
 // small group of heads only pads N to 8 or 16): S^T = K Q^T, an online
 // softmax per head column, then O^T += V^T P^T where movmatrix turns the
 // S^T accumulator fragment into the B operand.  The window branch reuses the
@@ -75,11 +75,20 @@ struct SpParams {
     unsigned long long wait_ns;
 };
 
-template <int NB>
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Gather the K and V rows of list entries [t0, t0+32) into `stage` and commit
+// them as one cp.async group.  Lane l validates entry t0+l; the 32 rows are
+// then copied two per instruction (16 lanes x 16 bytes per 256-byte row).
 __device__ __forceinline__ void issue_chunk(const SpParams &p, const int32_t *list, bool from_list, int lo,
                                             int n_list, int t0, int pos, const __nv_bfloat16 *kb,
-                                            const __nv_bfloat16 *vb, uint8_t *stage, uint32_t bar,
-                                            uint32_t &vmask, int lane) {
+                                            const __nv_bfloat16 *vb, uint8_t *stage, uint32_t &vmask, int lane) {
     const int t = t0 + lane;
     int key = -1;
     if (t < n_list) {
@@ -89,24 +98,20 @@ __device__ __forceinline__ void issue_chunk(const SpParams &p, const int32_t *li
             key = -1;
         }
     }
-    const bool valid = key >= 0;
-    vmask = __ballot_sync(0xffffffffu, valid);
-    if (lane == 0) mbar_expect_tx(bar, (uint32_t)__popc(vmask) * 512u);
-    __syncwarp();
-    uint8_t *krow = stage + lane * RS;
-    uint8_t *vrow = stage + CH * RS + lane * RS;
-    if (valid) {
-        const size_t ro = (size_t)key * p.Hkv * 128;
-        bulk_g2s(smem_u32(krow), kb + ro, 256, bar);
-        bulk_g2s(smem_u32(vrow), vb + ro, 256, bar);
-    } else {
-        const uint4 z = make_uint4(0, 0, 0, 0);
+    vmask = __ballot_sync(0xffffffffu, key >= 0);
+    const uint32_t sbase = smem_u32(stage);
+    const int half = lane >> 4, part = lane & 15;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            reinterpret_cast<uint4 *>(krow)[c] = z;
-            reinterpret_cast<uint4 *>(vrow)[c] = z;
-        }
+    for (int r2 = 0; r2 < CH / 2; ++r2) {
+        const int row = 2 * r2 + half;
+        const int kr = __shfl_sync(0xffffffffu, key, row);
+        const bool ok = kr >= 0;
+        const size_t so = ok ? (size_t)kr * p.Hkv * 128 + part * 8 : 0;
+        const uint32_t d = sbase + row * RS + part * 16;
+        cp_async16(d, kb + so, ok);
+        cp_async16(d + CH * RS, vb + so, ok);
     }
+    cp_async_commit();
 }
 
 template <int NB>
@@ -207,57 +212,55 @@ struct WarpCtx {
     const int32_t *list;
     const __nv_bfloat16 *kb, *vb;
     uint8_t *wbase;
-    uint32_t bar0;
     int lo, pos, lane;
     float c2;
 };
 
-__device__ __forceinline__ uint32_t pick3(uint32_t s, uint32_t a, uint32_t b, uint32_t c) {
+__device__ __forceinline__ uint32_t pick3(int s, uint32_t a, uint32_t b, uint32_t c) {
     return s == 0 ? a : (s == 1 ? b : c);
 }
 
 // Run one branch (from_list: the top-k list, else the causal window) through
-// the ST-stage gather pipeline.  `seq` counts chunks issued by this warp so
-// far (it fixes each stage's mbarrier parity).  Returns false on abort.
+// the ST-stage cp.async pipeline.  One group is committed per iteration (an
+// empty one past the end), so waiting for "at most ST-1 pending" always means
+// the chunk about to be used has landed.
 template <int NB>
-__device__ __forceinline__ bool run_branch(const WarpCtx &w, bool from_list, const uint32_t (&bq)[NB][8][2],
-                                           Branch<NB> &br, uint32_t &seq, int &aborted) {
+__device__ __forceinline__ void run_branch(const WarpCtx &w, bool from_list, const uint32_t (&bq)[NB][8][2],
+                                           Branch<NB> &br) {
     static_assert(ST == 3, "pick3 assumes three stages");
     const SpParams &p = *w.p;
     br.init();
     const int n_list = from_list ? p.topk : w.pos - w.lo + 1;
     const int nch = (n_list + CH - 1) / CH;
-    const uint32_t base = seq;
     uint32_t vm0 = 0, vm1 = 0, vm2 = 0;
     auto issue = [&](int c) {
-        const uint32_t sq_ = base + c, s = sq_ % ST;
-        uint32_t vmask;
-        issue_chunk<NB>(p, w.list, from_list, w.lo, n_list, c * CH, w.pos, w.kb, w.vb, w.wbase + s * STAGE_BYTES,
-                        w.bar0 + 8 * s, vmask, w.lane);
+        const int s = c % ST;
+        uint32_t vmask = 0;
+        if (c < nch) {
+            issue_chunk(p, w.list, from_list, w.lo, n_list, c * CH, w.pos, w.kb, w.vb, w.wbase + s * STAGE_BYTES,
+                        vmask, w.lane);
+        } else {
+            cp_async_commit();
+        }
         if (s == 0) vm0 = vmask; else if (s == 1) vm1 = vmask; else vm2 = vmask;
-        seq = sq_ + 1;
     };
-    const int pre = min(ST - 1, nch);
-    for (int c = 0; c < pre; ++c) issue(c);
+    for (int c = 0; c < ST - 1; ++c) issue(c);
 #pragma unroll 1
     for (int c = 0; c < nch; ++c) {
         __syncwarp();
-        if (c + ST - 1 < nch) issue(c + ST - 1);
-        const uint32_t sq_ = base + c, s = sq_ % ST;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(w.bar0 + 8 * s, (sq_ / ST) & 1, p.wait_ns, &aborted));
-        if (!ok) {
-            aborted = 1;
-            return false;
-        }
+        issue(c + ST - 1);
+        cp_async_wait<ST - 1>();
+        __syncwarp();
+        const int s = c % ST;
         compute_chunk<NB>(w.wbase + s * STAGE_BYTES, pick3(s, vm0, vm1, vm2), bq, w.c2, br, w.lane);
     }
-    return true;
+    cp_async_wait<0>();
+    __syncwarp();
 }
 
 template <int NB>
 __global__ void __launch_bounds__(SW * 32, 1) sparse_attn_mma(const SpParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t bars[SW][ST];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long item = (long long)blockIdx.x * SW + warp;
     if (item >= (long long)p.B * p.Lq * p.Hkv) return;   // whole warp leaves together
@@ -269,12 +272,6 @@ __global__ void __launch_bounds__(SW * 32, 1) sparse_attn_mma(const SpParams p) 
     const int pos = p.Lkv - p.Lq + i;
     uint8_t *wbase = smem + warp * SpSmem<NB>::WARP_BYTES;
     uint8_t *qs = wbase + ST * STAGE_BYTES;
-    const uint32_t bar0 = smem_u32(&bars[warp][0]);
-    if (lane == 0) {
-#pragma unroll
-        for (int s = 0; s < ST; ++s) mbar_init(bar0 + 8 * s, 1);
-        fence_mbar_init();
-    }
     // stage the group's query rows (zero rows pad the heads up to 8*NB)
     const size_t qrow = ((size_t)b * p.Lq + i) * p.Hq + (size_t)g * G;
     for (int e = lane; e < 8 * NB * 16; e += 32) {
@@ -298,25 +295,13 @@ __global__ void __launch_bounds__(SW * 32, 1) sparse_attn_mma(const SpParams p) 
     w.vb = p.v + ((size_t)b * p.Lkv * p.Hkv + g) * 128;
     w.list = p.idx + (((size_t)b * p.Hkv + g) * p.Lq + i) * p.topk;
     w.wbase = wbase;
-    w.bar0 = bar0;
     w.lo = max(0, pos - p.window + 1);
     w.pos = pos;
     w.lane = lane;
     w.c2 = p.scale_log2;
-    int aborted = 0;
-    uint32_t seq = 0;
     Branch<NB> bg, bl;
-    bool ok = run_branch<NB>(w, true, bq, bg, seq, aborted);
-    if (ok) ok = run_branch<NB>(w, false, bq, bl, seq, aborted);
-    if (!ok) {
-        // let every copy this warp issued land before the warp exits
-        for (uint32_t sq_ = seq > ST ? seq - ST : 0; sq_ < seq; ++sq_) {
-            int dummy = 0;
-            mbar_wait(bar0 + 8 * (sq_ % ST), (sq_ / ST) & 1, 1000000000ull, &dummy);
-        }
-        if (lane == 0) report(p.status, HS_ERR_TIMEOUT);
-        return;
-    }
+    run_branch<NB>(w, true, bq, bg);
+    run_branch<NB>(w, false, bq, bl);
 
     // gate merge, stage the G output rows in shared memory, write them once
     __syncwarp();
