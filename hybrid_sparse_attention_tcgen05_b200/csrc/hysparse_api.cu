@@ -6,6 +6,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "hysparse.h"
 #include "internal.h"
@@ -247,3 +249,68 @@ const char *hysparse_status_string(int status) {
 const char *hysparse_version(void) { return "hysparse-b200 0.1"; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of hysparse_full_attn_scores.
+//
+// Some callers cannot hand the library a workspace: code that runs after a
+// serving process has fixed its device memory (every later cudaMalloc is
+// refused or would break a memory budget the host framework enforces), and
+// hosts that give a plug-in only its input and output buffers and no way to
+// allocate.  For them this entry point keeps its scratch -- the status word
+// and the full layer's per-row softmax statistics -- in the fixed array
+// below, which every GPU that loads the library holds until the process
+// exits.  Host code may not use the array's name as a device address; the
+// address is looked up once per device with cudaGetSymbolAddress.
+namespace hs {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 16u << 20;  // 16 MiB
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 128;
+void *g_noalloc_ptr[kNoAllocMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device (set up on the
+// first call per device); nullptr and the CUDA error on failure.
+void *noalloc_scratch(cudaError_t *err) {
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess) return nullptr;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *ptr = nullptr;
+        *err = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (*err != cudaSuccess) return nullptr;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+}  // namespace hs
+
+extern "C" int hysparse_full_attn_scores_noalloc(const hs_shape *shape, const void *q, const void *k,
+                                                 const void *v, void *out, float *lse, float *scores,
+                                                 long long ld_scores, int row_begin, int row_count,
+                                                 hs_stream_t stream) {
+    Shape s;
+    int rc = resolve_shape(shape, &s);
+    if (rc != HS_OK) return rc;
+    rc = check_full_args(s, q, k, v, out, lse, scores, ld_scores, row_begin, row_count);
+    if (rc != HS_OK) return rc;
+    if (ws_layout(s, 1, row_count).stats_end > kNoAllocScratchBytes) return HS_ERR_WORKSPACE;
+    cudaError_t err = cudaSuccess;
+    void *ws = noalloc_scratch(&err);
+    if (ws == nullptr) return HS_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    // the status word must start at zero; the statistics are written before
+    // they are read, so the rest of the array is left as the last call left it
+    if (cudaMemsetAsync(ws, 0, kStatusBytes, st) != cudaSuccess) return HS_ERR_CUDA;
+    return run_full(s, q, k, v, out, lse, scores, ld_scores, row_begin, row_count, ws, st);
+}

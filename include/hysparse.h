@@ -143,6 +143,32 @@ int hysparse_block(const hs_shape *shape, const void *q_full, const void *k, con
                    const float *const *gate_logit, void *const *out_sparse, int topk, int window,
                    int32_t *idx_out, int row_chunk, void *ws, size_t ws_bytes, hs_stream_t stream);
 
+/* Allocation-free variant of hysparse_full_attn_scores (the pages have no
+ * counterpart; this is a deployment convenience).  Same computation,
+ * arguments, layouts and errors, but no workspace: its scratch (a status
+ * word and the per-row softmax statistics, 256 + 8*B*Hq*Lq bytes rounded up
+ * to 256) lives in a fixed 16 MiB device array inside the library, so callers
+ * that may not allocate device memory -- a serving process that has frozen
+ * its memory pool, or a plug-in host that only lends input and output
+ * buffers -- can still run the full layer.  Every GPU that loads the library
+ * holds that array until the process exits.
+ *   - Shapes whose scratch exceeds 16 MiB return HS_ERR_WORKSPACE (score
+ *     smaller row chunks or use hysparse_full_attn_scores instead).
+ *   - Calls no cudaMalloc/cudaFree and allocates nothing; the caller still
+ *     provides q, k, v, out, lse and (optionally) scores.
+ *   - The array's device address is looked up on the first call on each
+ *     device (the current device, which `stream` must belong to); make that
+ *     first call before any stream capture.
+ *   - All calls share the one array and each zeroes its status word on
+ *     `stream`: calls that can overlap on the GPU (other streams, other host
+ *     threads without ordering) race on it and must be serialised by the
+ *     caller.  Device-side timeouts are recorded there but are not readable
+ *     through this API. */
+int hysparse_full_attn_scores_noalloc(const hs_shape *shape, const void *q, const void *k,
+                                      const void *v, void *out, float *lse, float *scores,
+                                      long long ld_scores, int row_begin, int row_count,
+                                      hs_stream_t stream);
+
 /* Synchronises `stream`, reads the workspace status word (HS_OK or the
  * lowest-numbered device error recorded since it was last cleared), clears
  * it and returns it.  Returns HS_ERR_CUDA if the synchronisation fails. */
