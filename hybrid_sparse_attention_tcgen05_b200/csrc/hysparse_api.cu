@@ -45,9 +45,12 @@ int resolve_shape(const hs_shape *in, Shape *out) {
 struct WsLayout {
     size_t status = 0;
     size_t stats = 0, stats_end = 0;          // full layer per-row statistics
+    size_t dec = 0, full_end = 0;             // decode split-K partials + logit stash
     size_t block_scores = 0, block_lse = 0, block_idx = 0;
     size_t total = 0;
 };
+
+bool use_decode_path(const Shape &s) { return s.Lq == 1 && sparse_mma_supported(s); }
 
 WsLayout ws_layout(const Shape &s, int topk, int row_chunk) {
     WsLayout L;
@@ -55,6 +58,9 @@ WsLayout ws_layout(const Shape &s, int topk, int row_chunk) {
     L.stats = off;
     off = align_up(off + (size_t)s.B * s.Hq * s.Lq * 2 * sizeof(float), 256);
     L.stats_end = off;
+    L.dec = off;
+    if (use_decode_path(s)) off = align_up(off + decode_ws_bytes(s), 256);
+    L.full_end = off;
     const int chunk = (row_chunk <= 0 || row_chunk > s.Lq) ? s.Lq : row_chunk;
     L.block_scores = off;
     off = align_up(off + (size_t)s.B * s.Hkv * chunk * (size_t)s.Lkv * sizeof(float), 256);
@@ -79,6 +85,12 @@ int check_full_args(const Shape &s, const void *q, const void *k, const void *v,
 
 int run_full(const Shape &s, const void *q, const void *k, const void *v, void *out, float *lse,
              float *scores, long long ld, int row_begin, int row_count, void *ws, cudaStream_t st) {
+    if (use_decode_path(s)) {
+        char *w = reinterpret_cast<char *>(ws);
+        unsigned int *status = reinterpret_cast<unsigned int *>(ws);
+        return cuda_status(decode_full_mma_launch(s, q, k, v, out, lse, scores, ld,
+                                                  w + ws_layout(s, 1, row_count).dec, status, st));
+    }
     if (full_attn_tc_supported(s) && s.Lq >= kTcMinRows) {
         char *w = reinterpret_cast<char *>(ws);
         float2 *stats = reinterpret_cast<float2 *>(w + ws_layout(s, 1, row_count).stats);
@@ -140,7 +152,7 @@ int hysparse_full_attn_scores(const hs_shape *shape, const void *q, const void *
     rc = check_full_args(s, q, k, v, out, lse, scores, ld_scores, row_begin, row_count);
     if (rc != HS_OK) return rc;
     if (!aligned16(ws)) return HS_ERR_INVALID_ARG;
-    if (ws_bytes < ws_layout(s, 1, row_count).stats_end) return HS_ERR_WORKSPACE;
+    if (ws_bytes < ws_layout(s, 1, row_count).full_end) return HS_ERR_WORKSPACE;
     return run_full(s, q, k, v, out, lse, scores, ld_scores, row_begin, row_count, ws,
                     (cudaStream_t)stream);
 }
@@ -304,7 +316,7 @@ extern "C" int hysparse_full_attn_scores_noalloc(const hs_shape *shape, const vo
     if (rc != HS_OK) return rc;
     rc = check_full_args(s, q, k, v, out, lse, scores, ld_scores, row_begin, row_count);
     if (rc != HS_OK) return rc;
-    if (ws_layout(s, 1, row_count).stats_end > kNoAllocScratchBytes) return HS_ERR_WORKSPACE;
+    if (ws_layout(s, 1, row_count).full_end > kNoAllocScratchBytes) return HS_ERR_WORKSPACE;
     cudaError_t err = cudaSuccess;
     void *ws = noalloc_scratch(&err);
     if (ws == nullptr) return HS_ERR_CUDA;

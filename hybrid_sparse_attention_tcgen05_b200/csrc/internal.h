@@ -42,6 +42,13 @@ cudaError_t sparse_attn_mma_launch(const Shape &s, const void *q, const void *k,
                                    void *og, void *ol, unsigned int *status, unsigned long long wait_ns,
                                    cudaStream_t st);
 
+// sparse_mma.cu, decode full layer (bf16, d = 128, G <= 16, Lq == 1): split-K
+// partials + logit stash in `ws` (decode_ws_bytes of it), then a combine.
+size_t decode_ws_bytes(const Shape &s);
+cudaError_t decode_full_mma_launch(const Shape &s, const void *q, const void *k, const void *v, void *out,
+                                   float *lse, float *scores, long long ld, void *ws, unsigned int *status,
+                                   cudaStream_t st);
+
 // Upper bound (ns) on any single barrier wait inside a kernel; after it the
 // kernel records HS_ERR_TIMEOUT in the workspace status word and returns.
 unsigned long long wait_limit_ns();

@@ -116,7 +116,8 @@ __device__ __forceinline__ void issue_chunk(const SpParams &p, const int32_t *li
 
 template <int NB>
 __device__ __forceinline__ void compute_chunk(const uint8_t *stage, uint32_t vmask, const uint32_t (&bq)[NB][8][2],
-                                              float c2, Branch<NB> &br, int lane) {
+                                              float c2, Branch<NB> &br, int lane, float *stash = nullptr,
+                                              long long stash_ld = 0, int j0 = 0, int G = 0) {
     const uint32_t ks_base = smem_u32(stage);
     const uint32_t vs_base = smem_u32(stage + CH * RS);
     float c[NB][2][4];
@@ -158,6 +159,11 @@ __device__ __forceinline__ void compute_chunk(const uint8_t *stage, uint32_t vma
                 for (int rh = 0; rh < 2; ++rh) {
                     x[mt][rh] = kv[mt][rh] ? c[nb][mt][2 * rh + e] * c2 : -INFINITY;
                     cm = fmaxf(cm, x[mt][rh]);
+                    if (stash != nullptr) {
+                        const int h = 8 * nb + 2 * (lane & 3) + e;
+                        if (h < G && kv[mt][rh])
+                            stash[(long long)h * stash_ld + j0 + 16 * mt + (lane >> 2) + 8 * rh] = x[mt][rh];
+                    }
                 }
             cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 4));
             cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 8));
@@ -214,6 +220,9 @@ struct WarpCtx {
     uint8_t *wbase;
     int lo, pos, lane;
     float c2;
+    float *stash = nullptr;   // decode full layer: scaled logits [G][stash_ld]
+    long long stash_ld = 0;
+    int G = 0;
 };
 
 __device__ __forceinline__ uint32_t pick3(int s, uint32_t a, uint32_t b, uint32_t c) {
@@ -252,7 +261,8 @@ __device__ __forceinline__ void run_branch(const WarpCtx &w, bool from_list, con
         cp_async_wait<ST - 1>();
         __syncwarp();
         const int s = c % ST;
-        compute_chunk<NB>(w.wbase + s * STAGE_BYTES, pick3(s, vm0, vm1, vm2), bq, w.c2, br, w.lane);
+        compute_chunk<NB>(w.wbase + s * STAGE_BYTES, pick3(s, vm0, vm1, vm2), bq, w.c2, br, w.lane, w.stash,
+                          w.stash_ld, w.lo + c * CH, w.G);
     }
     cp_async_wait<0>();
     __syncwarp();
@@ -345,6 +355,147 @@ __global__ void __launch_bounds__(SW * 32, 1) sparse_attn_mma(const SpParams p) 
     }
 }
 
+// ------------------------------------------------------------ decode full layer
+//
+// One new query row per batch element (Lq = 1): the full layer is a stream
+// over the whole cache, bound by HBM.  Split-K: one warp owns (batch, KV head,
+// chunk of kDecChunk keys) and runs the contiguous-range pipeline above,
+// writing its online-softmax partial (m, l, unnormalised O per head) and the
+// scaled logits of every key (the stash).  decode_combine then merges the
+// partials into O and LSE and turns the stash into the exact group-summed
+// probabilities with the final per-head max and sum.
+
+constexpr int kDecChunk = 1024;
+
+struct DecParams {
+    SpParams sp;
+    float *part_o;      // [B][Hq][nchunk][128]
+    float2 *part_ml;    // [B][Hq][nchunk]  (m in log2 units, l)
+    float *stash;       // [B][Hq][Lkv]
+    int nchunk;
+};
+
+template <int NB>
+__global__ void __launch_bounds__(SW * 32, 1) decode_full_mma(const DecParams dp) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const SpParams &p = dp.sp;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long item = (long long)blockIdx.x * SW + warp;
+    if (item >= (long long)p.B * p.Hkv * dp.nchunk) return;
+    const int ch = (int)(item % dp.nchunk);
+    const long long bg = item / dp.nchunk;
+    const int g = (int)(bg % p.Hkv);
+    const int b = (int)(bg / p.Hkv);
+    const int G = p.G;
+    uint8_t *wbase = smem + warp * SpSmem<NB>::WARP_BYTES;
+    uint8_t *qs = wbase + ST * STAGE_BYTES;
+    const size_t qrow = (size_t)b * p.Hq + (size_t)g * G;      // Lq == 1
+    for (int e = lane; e < 8 * NB * 16; e += 32) {
+        const int h = e >> 4, cc = e & 15;
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (h < G) val = __ldg(reinterpret_cast<const uint4 *>(p.q + (qrow + h) * 128) + cc);
+        *reinterpret_cast<uint4 *>(qs + h * RS + cc * 16) = val;
+    }
+    __syncwarp();
+    uint32_t bq[NB][8][2];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int kp = 0; kp < 4; ++kp)
+            ldsm_x4(smem_u32(qs + (8 * nb + (lane & 7)) * RS + (32 * kp + 8 * (lane >> 3)) * 2),
+                    bq[nb][2 * kp][0], bq[nb][2 * kp][1], bq[nb][2 * kp + 1][0], bq[nb][2 * kp + 1][1]);
+    const int lo = ch * kDecChunk;
+    const int hi = min(p.Lkv, lo + kDecChunk);
+    WarpCtx w;
+    w.p = &p;
+    w.kb = p.k + ((size_t)b * p.Lkv * p.Hkv + g) * 128;
+    w.vb = p.v + ((size_t)b * p.Lkv * p.Hkv + g) * 128;
+    w.list = nullptr;
+    w.wbase = wbase;
+    w.lo = lo;
+    w.pos = hi - 1;            // the range [lo, hi) is read as a "window" ending at hi-1
+    w.lane = lane;
+    w.c2 = p.scale_log2;
+    w.stash = dp.stash + qrow * (size_t)p.Lkv;
+    w.stash_ld = p.Lkv;
+    w.G = G;
+    Branch<NB> br;
+    run_branch<NB>(w, false, bq, br);
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int h = 8 * nb + 2 * (lane & 3) + e;
+            if (h >= G) continue;
+            const size_t pi = (qrow + h) * dp.nchunk + ch;
+            if ((lane >> 2) == 0) dp.part_ml[pi] = make_float2(br.m[nb][e], br.l[nb][e]);
+            float *po = dp.part_o + pi * 128;
+#pragma unroll
+            for (int md = 0; md < 8; ++md)
+#pragma unroll
+                for (int rh = 0; rh < 2; ++rh) po[16 * md + (lane >> 2) + 8 * rh] = br.o[nb][md][2 * rh + e];
+        }
+}
+
+// One CTA per (batch, KV head): merge the split-K partials of the G heads
+// into O and LSE, then write the importance row from the logit stash.
+__global__ void __launch_bounds__(256) decode_combine(const DecParams dp, float *lse, float *scores,
+                                                      long long ld_scores) {
+    const SpParams &p = dp.sp;
+    const int g = blockIdx.x, b = blockIdx.y;
+    const int G = p.G;
+    __shared__ float s_m[32], s_il[32];
+    const size_t qrow = (size_t)b * p.Hq + (size_t)g * G;
+    for (int h = threadIdx.x >> 7; h < G; h += blockDim.x >> 7) {
+        const int d = threadIdx.x & 127;
+        const float2 *ml = dp.part_ml + (qrow + h) * dp.nchunk;
+        float M = -INFINITY;
+        for (int c = 0; c < dp.nchunk; ++c) M = fmaxf(M, ml[c].x);
+        float L = 0.f, acc = 0.f;
+        const float *po = dp.part_o + (qrow + h) * dp.nchunk * 128;
+        for (int c = 0; c < dp.nchunk; ++c) {
+            const float2 v = ml[c];
+            const float f = v.x == -INFINITY ? 0.f : ex2f(v.x - M);
+            L = fmaf(v.y, f, L);
+            acc = fmaf(po[(size_t)c * 128 + d], f, acc);
+        }
+        p.out[(qrow + h) * 128 + d] = __float2bfloat16_rn(acc / L);
+        if (d == 0) {
+            lse[qrow + h] = (M + log2f(L)) * kLn2;
+            s_m[h] = M;
+            s_il[h] = 1.0f / L;
+        }
+    }
+    __syncthreads();
+    if (scores == nullptr) return;
+    const float *st = dp.stash + qrow * (size_t)p.Lkv;
+    float *srow = scores + ((size_t)b * p.Hkv + g) * ld_scores;
+    for (int j = threadIdx.x; j < p.Lkv; j += blockDim.x) {
+        float sc = 0.f;
+        for (int h = 0; h < G; ++h) sc = fmaf(ex2f(st[(size_t)h * p.Lkv + j] - s_m[h]), s_il[h], sc);
+        srow[j] = sc;
+    }
+}
+
+template <int NB>
+cudaError_t launch_decode(const DecParams &dp, float *lse, float *scores, long long ld, cudaStream_t st) {
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(decode_full_mma<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SpSmem<NB>::bytes);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    const long long items = (long long)dp.sp.B * dp.sp.Hkv * dp.nchunk;
+    const long long blocks = (items + SW - 1) / SW;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+    decode_full_mma<NB><<<(unsigned)blocks, SW * 32, SpSmem<NB>::bytes, st>>>(dp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    decode_combine<<<dim3(dp.sp.Hkv, dp.sp.B), 256, 0, st>>>(dp, lse, scores, ld);
+    return cudaGetLastError();
+}
+
 template <int NB>
 cudaError_t launch_nb(const SpParams &p, cudaStream_t st) {
     static bool attr = false;
@@ -374,6 +525,32 @@ cudaError_t sparse_attn_mma_launch(const Shape &s, const void *q, const void *k,
                    (__nv_bfloat16 *)out, (__nv_bfloat16 *)og, (__nv_bfloat16 *)ol, s.B, s.Lq, s.Lkv, s.Hq,
                    s.Hkv, s.G(), topk, window, s.scale * kLog2e, status, wait_ns};
     return s.G() <= 8 ? tc::launch_nb<1>(p, st) : tc::launch_nb<2>(p, st);
+}
+
+size_t decode_ws_bytes(const Shape &s) {
+    const size_t nchunk = (s.Lkv + tc::kDecChunk - 1) / tc::kDecChunk;
+    const size_t rows = (size_t)s.B * s.Hq;
+    return rows * nchunk * 128 * sizeof(float) + rows * nchunk * sizeof(float2) + rows * s.Lkv * sizeof(float) +
+           3 * 256;
+}
+
+cudaError_t decode_full_mma_launch(const Shape &s, const void *q, const void *k, const void *v, void *out,
+                                   float *lse, float *scores, long long ld, void *ws, unsigned int *status,
+                                   cudaStream_t st) {
+    const int nchunk = (s.Lkv + tc::kDecChunk - 1) / tc::kDecChunk;
+    const size_t rows = (size_t)s.B * s.Hq;
+    char *w = reinterpret_cast<char *>(ws);
+    tc::DecParams dp;
+    dp.sp = tc::SpParams{(const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, nullptr,
+                         nullptr, (__nv_bfloat16 *)out, nullptr, nullptr, s.B, 1, s.Lkv, s.Hq, s.Hkv, s.G(),
+                         1, 1, s.scale * kLog2e, status, 0};
+    dp.part_o = reinterpret_cast<float *>(w);
+    w += align_up(rows * nchunk * 128 * sizeof(float), 256);
+    dp.part_ml = reinterpret_cast<float2 *>(w);
+    w += align_up(rows * nchunk * sizeof(float2), 256);
+    dp.stash = reinterpret_cast<float *>(w);
+    dp.nchunk = nchunk;
+    return s.G() <= 8 ? tc::launch_decode<1>(dp, lse, scores, ld, st) : tc::launch_decode<2>(dp, lse, scores, ld, st);
 }
 
 }  // namespace hs

@@ -159,6 +159,8 @@ SWEEP = [
     ("bf16_g16", 1, 200, 260, 32, 2, 128, "bf16", 100, 17, "shifted"),
     ("bf16_g1_ragged", 2, 129, 129, 2, 2, 128, "bf16", 1, 3, "normal"),
     ("bf16_decode", 4, 1, 1000, 32, 8, 128, "bf16", 128, 128, "normal"),
+    ("bf16_decode_multichunk_g16", 3, 1, 2500, 32, 2, 128, "bf16", 200, 128, "normal"),
+    ("bf16_decode_shifted_g4", 2, 1, 4097, 16, 4, 128, "bf16", 512, 128, "shifted"),
     ("bf16_window_ge_len", 1, 130, 130, 4, 1, 128, "bf16", 16, 1024, "shifted"),
 ]
 
