@@ -330,14 +330,23 @@ def bench_ours(args, w, ws_, rank, local):
     wm = work_model(w)
     per = {kk: vv / args.steps for kk, vv in stage_ms.items()}
     dom = max(per, key=per.get)
-    if dom == "full":
+    if dom == "full" and w.Lq == 1:
+        # decode: one new row per sequence streams the whole cache -> HBM bound
+        launches = n_chunks
+        dur_s = per["full"] / launches / 1e3
+        achieved = wm["kv_bytes"] / dur_s / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"kernel": "decode_full_mma+decode_combine", "bound": "hbm", "unit": "GB/s",
+                "work": "K and V of every (batch, KV head) read once: 2*B*Lkv*Hkv*d*2 bytes"}
+        key, srcs = "decode_full", ("sparse_mma.cu",)
+    elif dom == "full":
         launches = n_chunks
         dur_s = per["full"] / launches / 1e3
         achieved = wm["flops_full_scores"] / n_chunks / dur_s / 1e12
         peak = peaks["bf16_tflops"]
         roof = {"kernel": "full_attn_scores", "bound": "tensor", "unit": "TFLOP/s",
                 "work": "6*d*Hq per causal pair (QK^T+PV forward, QK^T score pass)"}
-        key, srcs = "full_attn_scores", ("simt_attn.cu",)
+        key, srcs = "full_attn_scores", ("attn_tc.cu",)
     elif dom == "topk":
         launches = n_chunks
         dur_s = per["topk"] / launches / 1e3
@@ -353,11 +362,20 @@ def bench_ours(args, w, ws_, rank, local):
         peak = peaks["hbm_gbs"]
         roof = {"kernel": "sparse_attn", "bound": "hbm", "unit": "GB/s",
                 "work": "(k_eff + w_eff) K and V rows per (row, kv head) + q, gate, out, idx"}
-        key, srcs = "sparse_attn", ("simt_attn.cu",)
+        key, srcs = "sparse_attn", ("sparse_mma.cu",)
     roof.update({"achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} (burst)",
                  "frac": achieved / peak, "launch_ms": dur_s * 1e3,
                  "traffic": read_traffic(key, source_hash(*srcs))})
-    gpu_launches = args.steps * (2 * n_chunks + w.n_sparse)
+    stage_ctx = {
+        "full": {"ms": per["full"], "tflops": (wm["flops_full_scores"] / (per["full"] / 1e3) / 1e12) if w.Lq > 1 else None,
+                 "hbm_gbs": (wm["kv_bytes"] / (per["full"] / 1e3) / 1e9) if w.Lq == 1 else None},
+        "topk": {"ms": per["topk"], "gbs": (wm["score_bytes"] / 2 + 4.0 * w.B * w.Hkv * w.Lq * w.topk)
+                 / (per["topk"] / 1e3) / 1e9},
+        "sparse_per_layer": {"ms": per["sparse"] / max(1, w.n_sparse),
+                             "gbs": wm["gather_bytes_per_layer"] / (per["sparse"] / max(1, w.n_sparse) / 1e3) / 1e9},
+    }
+    full_launches = n_chunks * (2 if w.dtype == "bf16" else 1)   # fwd+scores or split-K+combine
+    gpu_launches = args.steps * (full_launches + n_chunks + w.n_sparse)
     res = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -375,6 +393,7 @@ def bench_ours(args, w, ws_, rank, local):
         "gpu_launches": gpu_launches,
         "roofline": roof,
         "stages_ms_per_step": per,
+        "stages": stage_ctx,
         "wall_s_timed": wall,
     }
     if w.Lq == 1:
