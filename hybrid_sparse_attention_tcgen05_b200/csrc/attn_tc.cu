@@ -33,61 +33,12 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc_attn.cuh"
 #include "tc_util.cuh"
 
 namespace hs {
 namespace tc {
 namespace {
-
-constexpr int BM = 128;                 // query rows per tile
-constexpr int BN = 128;                 // keys per tile
-constexpr int HD = 128;                 // head dim
-constexpr int TILE = BM * HD * 2;       // one 128x128 bf16 tile: 32 KB
-constexpr int HALF = TILE / 2;          // one 64-column swizzled half: 16 KB
-constexpr int KV_STAGES = 4;
-constexpr int FWD_THREADS = 320;
-constexpr uint64_t kDrainNs = 1000000000ull;
-
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
-    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-// Wait that ignores the abort flag: used only to drain our own in-flight
-// copies / MMAs before the CTA exits.
-__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
-    int dummy = 0;
-    mbar_wait(bar, parity, kDrainNs, &dummy);
-}
-
-// S = Q K^T for one 128x128 tile: 8 MMAs of K=16 along the head dim.  Both
-// operands are K-major 128-byte-swizzled [128][64] halves 16 KB apart.
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
-    constexpr uint32_t I = idesc_bf16(128, 128, false, false);
-#pragma unroll
-    for (int kk = 0; kk < HD / 16; ++kk) {
-        const uint32_t o = (kk >> 2) * HALF + (kk & 3) * 32;
-        mma_ss(d_tmem, sdesc_sw128(q_addr + o, 16, 1024), sdesc_sw128(k_addr + o, 16, 1024), I,
-               kk > 0 ? 1u : 0u);
-    }
-}
-
-// O (+)= P V: P is 128x128 bf16 in TMEM (64 columns), V a [128 keys][128 d]
-// tile stored as two [128][64] swizzled halves -> N(=d)-major B operand.
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr,
-                                         bool accumulate) {
-    constexpr uint32_t I = idesc_bf16(128, 128, false, true);
-#pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk) {
-        mma_ts(d_tmem, p_tmem + kk * 8, sdesc_sw128(v_addr + kk * 2048, HALF, 1024), I,
-               (accumulate || kk > 0) ? 1u : 0u);
-    }
-}
 
 struct FwdBars {
     uint64_t q_full;
@@ -548,33 +499,6 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
 }
 
 // ----------------------------------------------------------------- host side
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
-// [B][L][H][128] bf16 -> 4-D map (d, H, L, B) with a {64, 1, 128, 1} box,
-// 128-byte swizzle; rows past L read as zeros.
-bool make_map(CUtensorMap *m, const void *base, int H, int L, int B) {
-    auto enc = encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
-    cuuint64_t strides[3] = {(cuuint64_t)HD * 2, (cuuint64_t)HD * 2 * H, (cuuint64_t)HD * 2 * H * L};
-    cuuint32_t box[4] = {64, 1, (cuuint32_t)BM, 1};
-    cuuint32_t es[4] = {1, 1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
 
 }  // namespace
 }  // namespace tc

@@ -46,6 +46,7 @@ struct WsLayout {
     size_t status = 0;
     size_t stats = 0, stats_end = 0;          // full layer per-row statistics
     size_t dec = 0, full_end = 0;             // decode split-K partials + logit stash
+    size_t selmask = 0, sparse_end = 0;       // dense-masked sparse layer: selection bitmask
     size_t block_scores = 0, block_lse = 0, block_idx = 0;
     size_t total = 0;
 };
@@ -61,6 +62,9 @@ WsLayout ws_layout(const Shape &s, int topk, int row_chunk) {
     L.dec = off;
     if (use_decode_path(s)) off = align_up(off + decode_ws_bytes(s), 256);
     L.full_end = off;
+    L.selmask = off;
+    if (sparse_dense_supported(s)) off = align_up(off + selmask_bytes(s), 256);
+    L.sparse_end = off;
     const int chunk = (row_chunk <= 0 || row_chunk > s.Lq) ? s.Lq : row_chunk;
     L.block_scores = off;
     off = align_up(off + (size_t)s.B * s.Hkv * chunk * (size_t)s.Lkv * sizeof(float), 256);
@@ -107,10 +111,42 @@ int run_topk(const Shape &s, const float *scores, long long ld, int row_begin, i
     return cuda_status(topk_launch(s, scores, ld, row_begin, row_count, topk, idx, st));
 }
 
+// Which sparse-layer kernel to run.  Both compute the same two softmaxes;
+// the estimate compares the dense-masked pass (every causal 128x128 tile of
+// every query head on the tensor cores, ~1500 cycles per tile on one SM) with
+// the gather (k_eff + w_eff K and V rows of 256 bytes per row and KV head at
+// ~6 TB/s).  HYSPARSE_SPARSE_PATH=dense|gather overrides it.
+bool prefer_dense_sparse(const Shape &s, int topk, int window) {
+    if (!sparse_dense_supported(s)) return false;
+    const char *e = getenv("HYSPARSE_SPARSE_PATH");
+    if (e && strcmp(e, "dense") == 0) return true;
+    if (e && strcmp(e, "gather") == 0) return false;
+    const double off = (double)(s.Lkv - s.Lq);
+    double tiles = 0.0;                       // sum over 128-row tiles of causal key tiles
+    const int n_rt = (s.Lq + 127) / 128;
+    for (int t = 0; t < n_rt; ++t) {
+        const double last = off + fmin((double)s.Lq, 128.0 * (t + 1)) - 1.0;
+        tiles += floor(last / 128.0) + 1.0;
+    }
+    const double dense_s = tiles * s.Hq * s.B * 1500.0 / (148.0 * 1.9e9);
+    double keys = 0.0;                         // sum over rows of k_eff + w_eff
+    for (int i = 0; i < s.Lq; i += 64) {
+        const double n = off + i + 1.0;
+        keys += 64.0 * (fmin(n, (double)topk) + fmin(n, (double)window));
+    }
+    const double gather_s = keys * s.Hkv * s.B * 512.0 / 6.0e12;
+    return dense_s < gather_s;
+}
+
 int run_sparse(const Shape &s, const void *q, const void *k, const void *v, const int32_t *idx,
                int topk, const float *gate, int window, void *out, void *og, void *ol, void *ws,
                cudaStream_t st) {
     unsigned int *status = reinterpret_cast<unsigned int *>(ws);
+    if (prefer_dense_sparse(s, topk, window)) {
+        uint32_t *mask = reinterpret_cast<uint32_t *>(reinterpret_cast<char *>(ws) + ws_layout(s, topk, 1).selmask);
+        return cuda_status(sparse_dense_tc_launch(s, q, k, v, idx, topk, gate, window, out, og, ol, mask,
+                                                  status, wait_limit_ns(), st));
+    }
     if (sparse_mma_supported(s))
         return cuda_status(sparse_attn_mma_launch(s, q, k, v, idx, topk, gate, window, out, og, ol, status,
                                                   wait_limit_ns(), st));
@@ -182,7 +218,7 @@ int hysparse_sparse_attn(const hs_shape *shape, const void *q, const void *k, co
         return HS_ERR_INVALID_ARG;
     if (topk < 1 || topk > kMaxTopk || window < 1 || window > kMaxWindow) return HS_ERR_INVALID_ARG;
     if (!aligned16(ws)) return HS_ERR_INVALID_ARG;
-    if (ws_bytes < ws_layout(s, topk, 1).stats_end) return HS_ERR_WORKSPACE;
+    if (ws_bytes < ws_layout(s, topk, 1).sparse_end) return HS_ERR_WORKSPACE;
     return run_sparse(s, q, k, v, idx, topk, gate_logit, window, out, out_global, out_local, ws,
                       (cudaStream_t)stream);
 }

@@ -49,6 +49,16 @@ cudaError_t decode_full_mma_launch(const Shape &s, const void *q, const void *k,
                                    float *lse, float *scores, long long ld, void *ws, unsigned int *status,
                                    cudaStream_t st);
 
+// sparse_tc.cu: dense-masked sparse layer (bf16, d = 128, Lq >= 64); its
+// selection bitmask (selmask_bytes) lives in the caller's workspace.
+bool sparse_dense_supported(const Shape &s);
+int selmask_words(const Shape &s);
+size_t selmask_bytes(const Shape &s);
+cudaError_t sparse_dense_tc_launch(const Shape &s, const void *q, const void *k, const void *v,
+                                   const int32_t *idx, int topk, const float *gate, int window, void *out,
+                                   void *og, void *ol, uint32_t *mask, unsigned int *status,
+                                   unsigned long long wait_ns, cudaStream_t st);
+
 // Upper bound (ns) on any single barrier wait inside a kernel; after it the
 // kernel records HS_ERR_TIMEOUT in the workspace status word and returns.
 unsigned long long wait_limit_ns();

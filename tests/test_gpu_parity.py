@@ -162,11 +162,35 @@ SWEEP = [
     ("bf16_decode_multichunk_g16", 3, 1, 2500, 32, 2, 128, "bf16", 200, 128, "normal"),
     ("bf16_decode_shifted_g4", 2, 1, 4097, 16, 4, 128, "bf16", 512, 128, "shifted"),
     ("bf16_window_ge_len", 1, 130, 130, 4, 1, 128, "bf16", 16, 1024, "shifted"),
+    ("bf16_prefix_ragged", 2, 200, 333, 8, 2, 128, "bf16", 40, 100, "normal"),
+    ("bf16_window_256", 1, 600, 600, 8, 4, 128, "bf16", 300, 256, "shifted"),
 ]
 
 
-@pytest.mark.parametrize("case", SWEEP, ids=lambda c: c[0])
-def test_shape_sweep_all_rows(case):
+@pytest.fixture
+def sparse_path(request, monkeypatch):
+    """Force one sparse-layer kernel (dense-masked tcgen05 or gather) for
+    the test; None keeps the library's own choice."""
+    if request.param is None:
+        monkeypatch.delenv("HYSPARSE_SPARSE_PATH", raising=False)
+    else:
+        monkeypatch.setenv("HYSPARSE_SPARSE_PATH", request.param)
+    return request.param
+
+
+def _sweep_params():
+    out = []
+    for c in SWEEP:
+        paths = [None]
+        if c[7] == "bf16" and c[2] >= 64:
+            paths = ["gather", "dense"]
+        for pth in paths:
+            out.append(pytest.param(c, pth, id=f"{c[0]}-{pth or 'auto'}"))
+    return out
+
+
+@pytest.mark.parametrize("case,sparse_path", _sweep_params(), indirect=["sparse_path"])
+def test_shape_sweep_all_rows(case, sparse_path):
     name, B, Lq, Lkv, Hq, Hkv, d, dt, topk, window, dist = case
     w = gen.Workload(name, B, Lq, Lkv, Hq, Hkv, d, dt, topk, window, 2, dist)
     cpu = gen.make_inputs(w, seed=3, device="cpu")
@@ -179,11 +203,14 @@ def test_shape_sweep_all_rows(case):
 
 # ------------------------------------------------- full-size, sampled rows
 
-FULL = ["prefill8k", "prefill32k", "moe64k"]
+FULL = [pytest.param("prefill8k", "gather", id="prefill8k-gather"),
+        pytest.param("prefill8k", "dense", id="prefill8k-dense"),
+        pytest.param("prefill32k", None, id="prefill32k-auto"),
+        pytest.param("moe64k", None, id="moe64k-auto")]
 
 
-@pytest.mark.parametrize("name", FULL)
-def test_full_size_prefill_sampled_rows(name):
+@pytest.mark.parametrize("name,sparse_path", FULL, indirect=["sparse_path"])
+def test_full_size_prefill_sampled_rows(name, sparse_path):
     w = gen.WORKLOADS[name]
     inp = gen.make_inputs(w, seed=0, device=DEV)
     chunk = 4096 if w.Lq > 8192 else w.Lq
