@@ -113,9 +113,12 @@ int run_topk(const Shape &s, const float *scores, long long ld, int row_begin, i
 
 // Which sparse-layer kernel to run.  Both compute the same two softmaxes;
 // the estimate compares the dense-masked pass (every causal 128x128 tile of
-// every query head on the tensor cores, ~1500 cycles per tile on one SM) with
-// the gather (k_eff + w_eff K and V rows of 256 bytes per row and KV head at
-// ~6 TB/s).  HYSPARSE_SPARSE_PATH=dense|gather overrides it.
+// every query head on the tensor cores; kDenseTileCycles per tile on one SM,
+// measured) with the gather (k_eff + w_eff K and V rows of 256 bytes per row
+// and KV head at kGatherBytesPerS, measured).
+// HYSPARSE_SPARSE_PATH=dense|gather overrides it.
+constexpr double kDenseTileCycles = 10000.0;
+constexpr double kGatherBytesPerS = 6.0e12;
 bool prefer_dense_sparse(const Shape &s, int topk, int window) {
     if (!sparse_dense_supported(s)) return false;
     const char *e = getenv("HYSPARSE_SPARSE_PATH");
@@ -128,13 +131,13 @@ bool prefer_dense_sparse(const Shape &s, int topk, int window) {
         const double last = off + fmin((double)s.Lq, 128.0 * (t + 1)) - 1.0;
         tiles += floor(last / 128.0) + 1.0;
     }
-    const double dense_s = tiles * s.Hq * s.B * 1500.0 / (148.0 * 1.9e9);
+    const double dense_s = tiles * s.Hq * s.B * kDenseTileCycles / (148.0 * 1.9e9);
     double keys = 0.0;                         // sum over rows of k_eff + w_eff
     for (int i = 0; i < s.Lq; i += 64) {
         const double n = off + i + 1.0;
         keys += 64.0 * (fmin(n, (double)topk) + fmin(n, (double)window));
     }
-    const double gather_s = keys * s.Hkv * s.B * 512.0 / 6.0e12;
+    const double gather_s = keys * s.Hkv * s.B * 512.0 / kGatherBytesPerS;
     return dense_s < gather_s;
 }
 
