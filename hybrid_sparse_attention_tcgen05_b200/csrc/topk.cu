@@ -2,118 +2,191 @@
 // patterns (write-up section 2.2: the global branch attends over the full
 // layer's TopK indices; baidu article "Top-K selection").
 //
-// Importance scores are sums of probabilities, so they are >= 0 and their
-// IEEE-754 bit patterns, read as uint32, sort in the same order as the
-// values.  Four 8-bit digit passes find the exact bit pattern T of the k-th
-// largest score and how many keys equal to T must be taken; a final pass in
-// ascending key order emits every key above T and the lowest-indexed keys
-// equal to T, which is exactly "largest scores, ties to the lower index",
-// already in ascending order.  Integer work only: the result is exact and
-// deterministic.
-#include <cub/block/block_scan.cuh>
-
+// Importance scores are sums of probabilities, so they are >= 0: the sign
+// bit is 0 and the other 31 bits, read as an unsigned integer, sort in the
+// same order as the values.  Three digit passes (bits 30-20, 19-10, 9-0) find
+// the exact bit pattern T of the k-th largest score and how many keys equal
+// to T must be taken; an ordered compaction then emits every key above T and
+// the lowest-indexed keys equal to T, which is exactly "largest scores, ties
+// to the lower index", already in ascending key order.  Integer work only:
+// the result is exact and deterministic.
+//
+// Rows whose causal length fits (kSmemKeys) are first copied into shared
+// memory, so only that one read touches L2/HBM; longer rows are re-read from
+// global memory each pass.  Histogram updates are aggregated per warp
+// (__match_any_sync): near-flat score rows put almost every key in one bin,
+// and unaggregated shared atomics on one address serialise.  The compaction
+// uses per-warp ballot counts and one scan over warps instead of block-wide
+// scans per element chunk.
 #include "common.cuh"
 #include "internal.h"
 
 namespace hs {
 namespace {
 
-template <int NT>
-__global__ void __launch_bounds__(NT)
-topk_radix_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv, int Hkv,
-                  int row_begin, int row_count, int topk, int32_t *__restrict__ idx) {
-    using Scan = cub::BlockScan<int, NT>;
-    __shared__ typename Scan::TempStorage scan_tmp;
-    __shared__ unsigned int hist[256];
-    __shared__ unsigned int sh_digit, sh_remaining;
+constexpr int NT = 512;
+constexpr int NW = NT / 32;
+constexpr int kSmemKeys = 24576;       // 96 KB of row cache
+constexpr int kHistBins = 2048;
 
-    const int r = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x;
+struct TopkShared {
+    unsigned int hist[kHistBins];
+    unsigned int sh_digit, sh_remaining;
+    int cnt_gt[NW], cnt_eq[NW];
+};
+
+__device__ __forceinline__ void hist_add(unsigned int *hist, bool take, unsigned int bin, int lane) {
+    const unsigned int key = take ? bin : (0x80000000u | (unsigned)lane);   // unmatched lanes stay alone
+    const unsigned int peers = __match_any_sync(0xffffffffu, key);
+    if (take && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (unsigned)__popc(peers));
+}
+
+template <bool SMEM>
+__global__ void __launch_bounds__(NT)
+topk_radix_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv, int Hkv, int row_begin,
+                  int row_count, int r_lo, int topk, int32_t *__restrict__ idx) {
+    extern __shared__ unsigned int row_cache[];
+    __shared__ TopkShared sh;
+
+    const int r = r_lo + blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int i = row_begin + r;
     const int n = Lkv - Lq + i + 1;
-    const unsigned int *u = reinterpret_cast<const unsigned int *>(
-        scores + (((size_t)b * Hkv + g) * row_count + r) * ld);
+    const unsigned int *gu =
+        reinterpret_cast<const unsigned int *>(scores + (((size_t)b * Hkv + g) * row_count + r) * ld);
     int32_t *o = idx + (((size_t)b * Hkv + g) * Lq + i) * (size_t)topk;
 
     if (n <= topk) {
         for (int t = tid; t < topk; t += NT) o[t] = t < n ? t : -1;
         return;
     }
+    const unsigned int *u = gu;
+    if (SMEM) {
+        for (int j = tid; j < n; j += NT) row_cache[j] = __ldg(gu + j);
+        __syncthreads();
+        u = row_cache;
+    }
+    const int n_pad = (n + 31) & ~31;
 
     unsigned int prefix = 0, mask = 0, remaining = (unsigned int)topk;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int t = tid; t < 256; t += NT) hist[t] = 0;
+    const int shifts[3] = {20, 10, 0};
+    const int widths[3] = {11, 10, 10};
+#pragma unroll 1
+    for (int ps = 0; ps < 3; ++ps) {
+        const int shift = shifts[ps];
+        const unsigned int nb = 1u << widths[ps];
+        for (int t = tid; t < (int)nb; t += NT) sh.hist[t] = 0;
         __syncthreads();
-        for (int j = tid; j < n; j += NT) {
-            const unsigned int x = u[j];
-            if ((x & mask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
+        for (int j = tid; j < n_pad; j += NT) {
+            const bool in = j < n;
+            const unsigned int x = in ? (SMEM ? u[j] : __ldg(u + j)) : 0u;
+            const bool take = in && (x & mask) == prefix;
+            hist_add(sh.hist, take, (x >> shift) & (nb - 1u), lane);
         }
         __syncthreads();
-        if (tid < 32) {
-            // lane covers digits 255-8*lane .. 255-8*lane-7 (descending order)
-            unsigned int c[8], tot = 0;
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                c[t] = hist[255 - (8 * tid + t)];
-                tot += c[t];
-            }
+        if (warp == 0) {
+            // lane covers bins nb-1-L*per .. nb-L*per-per (descending)
+            const int per = (int)nb / 32;
+            unsigned int tot = 0;
+            for (int t = 0; t < per; ++t) tot += sh.hist[nb - 1 - (lane * per + t)];
             unsigned int incl = tot;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const unsigned int y = __shfl_up_sync(0xffffffffu, incl, off);
-                if (tid >= off) incl += y;
+                if (lane >= off) incl += y;
             }
             const unsigned int excl = incl - tot;
             if (excl < remaining && remaining <= incl) {
                 unsigned int cum = excl;
-#pragma unroll
-                for (int t = 0; t < 8; ++t) {
-                    if (cum + c[t] >= remaining) {
-                        sh_digit = 255u - (unsigned int)(8 * tid + t);
-                        sh_remaining = remaining - cum;
+                for (int t = 0; t < per; ++t) {
+                    const unsigned int c = sh.hist[nb - 1 - (lane * per + t)];
+                    if (cum + c >= remaining) {
+                        sh.sh_digit = nb - 1 - (unsigned)(lane * per + t);
+                        sh.sh_remaining = remaining - cum;
                         break;
                     }
-                    cum += c[t];
+                    cum += c;
                 }
             }
         }
         __syncthreads();
-        prefix |= sh_digit << shift;
-        mask |= 255u << shift;
-        remaining = sh_remaining;
+        prefix |= sh.sh_digit << shift;
+        mask |= (nb - 1u) << shift;
+        remaining = sh.sh_remaining;
         __syncthreads();
     }
 
-    // prefix == bit pattern of the k-th largest score; take every key above it
-    // and the first `remaining` keys equal to it, in ascending key order.
-    int base_sel = 0, base_eq = 0;
-    for (int j0 = 0; j0 < n; j0 += NT) {
-        const int j = j0 + tid;
-        const bool valid = j < n;
-        const unsigned int x = valid ? u[j] : 0u;
-        const int is_eq = (valid && x == prefix) ? 1 : 0;
-        int eq_rank, eq_total;
-        Scan(scan_tmp).ExclusiveSum(is_eq, eq_rank, eq_total);
-        __syncthreads();
-        const int sel = (valid && (x > prefix || (is_eq && base_eq + eq_rank < (int)remaining))) ? 1 : 0;
-        int sel_rank, sel_total;
-        Scan(scan_tmp).ExclusiveSum(sel, sel_rank, sel_total);
-        __syncthreads();
-        if (sel && base_sel + sel_rank < topk) o[base_sel + sel_rank] = j;
-        base_sel += sel_total;
-        base_eq += eq_total;
-        if (base_sel >= topk) break;
+    // prefix == the bit pattern of the k-th largest score.  Ordered
+    // compaction: warp w owns the contiguous key range [w*seg, (w+1)*seg).
+    // (A negative input, which importance scores never are, could only make
+    // more keys compare above T; the `at < topk` guard keeps writes in bounds.)
+    const unsigned int T = prefix;
+    const int seg = ((n + NW - 1) / NW + 31) & ~31;
+    const int j_lo = warp * seg, j_hi = min(n, j_lo + seg);
+    int gt = 0, eq = 0;
+    for (int j0 = j_lo; j0 < j_hi; j0 += 32) {
+        const int j = j0 + lane;
+        const unsigned int x = j < j_hi ? (SMEM ? u[j] : __ldg(u + j)) : 0u;
+        gt += __popc(__ballot_sync(0xffffffffu, j < j_hi && x > T));
+        eq += __popc(__ballot_sync(0xffffffffu, j < j_hi && x == T));
+    }
+    if (lane == 0) {
+        sh.cnt_gt[warp] = gt;
+        sh.cnt_eq[warp] = eq;
+    }
+    __syncthreads();
+    int gt_base = 0, eq_base = 0;
+    for (int w = 0; w < warp; ++w) {
+        gt_base += sh.cnt_gt[w];
+        eq_base += sh.cnt_eq[w];
+    }
+    const unsigned int lt_mask = (1u << lane) - 1u;
+    for (int j0 = j_lo; j0 < j_hi; j0 += 32) {
+        const int j = j0 + lane;
+        const unsigned int x = j < j_hi ? (SMEM ? u[j] : __ldg(u + j)) : 0u;
+        const unsigned int bg = __ballot_sync(0xffffffffu, j < j_hi && x > T);
+        const unsigned int be = __ballot_sync(0xffffffffu, j < j_hi && x == T);
+        const int gtb = gt_base + __popc(bg & lt_mask);
+        const int eqb = eq_base + __popc(be & lt_mask);
+        const bool is_gt = (bg >> lane) & 1u, is_eq = (be >> lane) & 1u;
+        if (is_gt || (is_eq && eqb < (int)remaining)) {
+            const int at = gtb + min(eqb, (int)remaining);
+            if (at < topk) o[at] = j;
+        }
+        gt_base += __popc(bg);
+        eq_base += __popc(be);
     }
 }
 
 }  // namespace
 
-cudaError_t topk_launch(const Shape &s, const float *scores, long long ld, int row_begin,
-                        int row_count, int topk, int32_t *idx, cudaStream_t st) {
-    constexpr int NT = 512;
-    dim3 grid(row_count, s.Hkv, s.B);
-    topk_radix_kernel<NT><<<grid, NT, 0, st>>>(scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count,
-                                                topk, idx);
+cudaError_t topk_launch(const Shape &s, const float *scores, long long ld, int row_begin, int row_count,
+                        int topk, int32_t *idx, cudaStream_t st) {
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kSmemKeys * 4);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    // rows are ordered by causal length; those up to kSmemKeys keys run with
+    // the row cached in shared memory, sized for the longest of them
+    const int off = s.Lkv - s.Lq;
+    const int n_first = off + row_begin + 1;
+    int split = row_count;                                   // rows [0, split) fit
+    if (n_first > kSmemKeys) split = 0;
+    else if (off + row_begin + row_count > kSmemKeys) split = kSmemKeys - off - row_begin;
+    if (split > 0) {
+        const int n_max = off + row_begin + split;
+        topk_radix_kernel<true><<<dim3(split, s.Hkv, s.B), NT, (size_t)n_max * 4, st>>>(
+            scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, 0, topk, idx);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (split < row_count) {
+        topk_radix_kernel<false><<<dim3(row_count - split, s.Hkv, s.B), NT, 0, st>>>(
+            scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, split, topk, idx);
+    }
     return cudaGetLastError();
 }
 

@@ -124,13 +124,18 @@ def test_topk_stage_isolated_bit_exact():
     assert torch.equal(idx[0, 0].cpu(), o_idx)
 
 
-@pytest.mark.parametrize("case", ["ties", "all_equal", "zeros_and_denormals", "long_rows"])
+@pytest.mark.parametrize("case", ["ties", "all_equal", "zeros_and_denormals", "long_rows", "split_rows",
+                                  "flat_narrow"])
 def test_topk_synthetic_rows_bit_exact(case):
     """Score rows built directly (not by the CUDA path), with exact ties."""
     g = torch.Generator().manual_seed(7)
     B, Hkv, Lq, Lkv, k = 2, 3, 37, 300, 29
     if case == "long_rows":
         Lq, Lkv, k = 5, 70000, 2048
+    elif case == "split_rows":      # rows on both sides of the shared-memory row-cache limit
+        Lq, Lkv, k = 40, 24600, 1000
+    elif case == "flat_narrow":     # near-flat rows: every key in one coarse bin
+        Lq, Lkv, k = 16, 20000, 1500
     s = torch.rand(B, Hkv, Lq, Lkv, generator=g)
     if case == "ties":
         s = torch.round(s * 16) / 16
@@ -140,6 +145,10 @@ def test_topk_synthetic_rows_bit_exact(case):
         s = torch.where(s < 0.5, torch.zeros_like(s), s * 1e-39)
     elif case == "long_rows":
         s = torch.round(s * 4096) / 4096
+    elif case == "split_rows":
+        s = torch.round(s * 65536) / 65536
+    elif case == "flat_narrow":
+        s = (1.0 + 0.02 * s) / 8192.0
     shape = hs.HsShape(B, Lq, Lkv, 4 * Hkv, Hkv, 128, 1, 0.0)
     idx = hs.topk(shape, s.to(DEV), k)
     n_valid = [Lkv - Lq + i + 1 for _ in range(B) for _ in range(Hkv) for i in range(Lq)]
