@@ -15,9 +15,9 @@
 // work differs.  The host picks this kernel or the gather kernel from a cost
 // estimate.
 //
-// CTA = 128 query rows of one query head.  Warps 0-7: softmax (two warps per
-// TMEM lane quarter, each on 64 of the 128 columns); warp 8: TMA producer (Q
-// once, then K_j, V_j through a 4-slot ring); warp 9: MMA issuer.  TMEM: S0 | S1 (double-buffered scores) | Og |
+// CTA = 128 query rows of one query head.  Warps 0-3: softmax (thread = row =
+// TMEM lane); warp 4: TMA producer (Q once, then K_j, V_j through a 4-slot
+// ring); warp 5: MMA issuer.  TMEM: S0 | S1 (double-buffered scores) | Og |
 // Ol.  P for the global branch overwrites S columns 0-63, P for the window
 // branch columns 64-127 (window tiles only); both feed PV MMAs from TMEM.
 #include <cuda.h>
@@ -31,7 +31,7 @@ namespace hs {
 namespace tc {
 namespace {
 
-constexpr int SD_THREADS = 320;   // warps 0-7 softmax, 8 TMA, 9 MMA
+constexpr int SD_THREADS = 192;
 constexpr int SD_KV = 4;
 
 struct SdBars {
@@ -58,14 +58,10 @@ struct SdParams {
     unsigned long long wait_ns;
 };
 
-__device__ __forceinline__ void named_bar(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// Rescale 64 columns of an accumulator row in TMEM by `corr` (per thread).
-__device__ __forceinline__ void tmem_scale64(uint32_t t, float corr) {
+// Rescale 128 columns of an accumulator row in TMEM by `corr` (per thread).
+__device__ __forceinline__ void tmem_scale128(uint32_t t, float corr) {
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
         tmem_ld32(t + 32 * c, o);
         tmem_wait_ld();
@@ -80,7 +76,6 @@ __global__ void __launch_bounds__(SD_THREADS, 1)
 sparse_dense_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const SdParams p) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ float sh_xch[2][4][128];   // [tile parity][half*2 + stream][row]
     uint8_t *smem = align1024(smem_raw);
     uint8_t *sq = smem;
     uint8_t *skv = smem + TILE;
@@ -107,7 +102,7 @@ sparse_dense_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
         }
         mbar_init(smem_u32(&bars->s_full[0]), 1);
         mbar_init(smem_u32(&bars->s_full[1]), 1);
-        mbar_init(smem_u32(&bars->p_full), 256);
+        mbar_init(smem_u32(&bars->p_full), 128);
         mbar_init(smem_u32(&bars->o_done), 1);
         mbar_init(smem_u32(&bars->o_final), 1);
         mbar_init(smem_u32(&bars->drain), 1);
@@ -124,7 +119,7 @@ sparse_dense_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     const uint32_t tmem = bars->tmem_base;
     volatile int *abort = &bars->abort;
 
-    if (warp == 8) {
+    if (warp == 4) {
         if (lane == 0) {
             tma_prefetch(&tq);
             tma_prefetch(&tk);
@@ -149,7 +144,7 @@ sparse_dense_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                     mbar_drain(smem_u32(&bars->kv_full[it % SD_KV]), (it / SD_KV) & 1);
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == 5) {
         if (lane == 0) {
             const uint32_t tS[2] = {tmem, tmem + 128};
             const uint32_t tOg = tmem + 256, tOl = tmem + 384;
@@ -188,152 +183,137 @@ sparse_dense_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             mbar_drain(smem_u32(&bars->drain), 0);
         }
     } else {
-        // softmax warps: warp w serves TMEM lanes 32*(w%4).. and S columns
-        // 64*(w/4) .. +63; the two warps of a lane quarter exchange row maxima
-        // (and, at the end, row sums) through shared memory.
-        const int q = warp & 3, half = warp >> 2;
-        const int tw = 32 * q + lane;
+        const int tw = threadIdx.x;
         const int row = r0 + tw;
         const bool valid = row < r_end;
         const int rrow = min(row, r_end - 1);
         const int pos = off + rrow;
         const int lo_w = max(0, pos - p.window + 1);
-        const uint32_t lane_off = (uint32_t)(32 * q) << 16;
-        const uint32_t colh = (uint32_t)(64 * half);
-        const uint32_t tOg = tmem + lane_off + 256u + colh, tOl = tmem + lane_off + 384u + colh;
-        const uint2 *mrow = reinterpret_cast<const uint2 *>(p.selmask + (((size_t)b * p.Hkv + g) * p.Lq + rrow) * p.W) + half;
+        const uint32_t lane_off = (uint32_t)(tw & ~31) << 16;
+        const uint32_t tOg = tmem + lane_off + 256u, tOl = tmem + lane_off + 384u;
+        const uint4 *mrow = reinterpret_cast<const uint4 *>(p.selmask + (((size_t)b * p.Hkv + g) * p.Lq + rrow) * p.W);
         const float c2 = p.scale_log2;
-        const int bar_id = 1 + q;
-        float mg = -INFINITY, lg = 0.f, ml = -INFINITY, ll = 0.f;
-        uint2 mw = __ldg(mrow);
-        bool live = true;
+        float mg = -INFINITY, lg = 0.f, cg = 0.f;
+        float ml = -INFINITY, ll = 0.f, cl = 0.f;
+        bool ok = true;
+        uint4 mw = __ldg(mrow);
         for (int j = 0; j < n_kv; ++j) {
             const int buf = j & 1;
             const uint32_t tS = tmem + lane_off + (uint32_t)(buf * 128);
-            const uint32_t mw0 = mw.x, mw1 = mw.y;
-            if (j + 1 < n_kv) mw = __ldg(mrow + 2 * (j + 1));   // next tile's 64 mask bits of this half
-            const int j0 = j * BN + 64 * half;                    // key index of column 0 of this half
-            const bool diag = j * BN + BN - 1 > pos_first;          // causal edge inside the tile (CTA-uniform)
-            const bool wtile = j >= jw0;
-            float s[64];
-            float mxg = -INFINITY, mxl = -INFINITY;
-            live = live && __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[buf]), (j >> 1) & 1, p.wait_ns, abort));
-            if (live) {
-                tc_fence_after();
-                uint32_t r[2][32];
-                tmem_ld32(tS + colh, r[0]);
-                tmem_ld32(tS + colh + 32, r[1]);
-                tmem_wait_ld();
-                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                float w4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            const uint32_t mwords[4] = {mw.x, mw.y, mw.z, mw.w};
+            if (j + 1 < n_kv) mw = __ldg(mrow + j + 1);   // prefetch the next tile's mask
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[buf]), (j >> 1) & 1, p.wait_ns, abort));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t r[4][32];
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    s[c] = __uint_as_float(r[c >> 5][c & 31]);
-                    bool sel = ((c < 32 ? mw0 : mw1) >> (c & 31)) & 1u;
-                    if (diag) sel = sel && (j0 + c <= pos);
-                    if (sel) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
-                    if (wtile && j0 + c >= lo_w && j0 + c <= pos) w4[c & 3] = fmaxf(w4[c & 3], s[c]);
-                }
-                mxg = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-                mxl = fmaxf(fmaxf(w4[0], w4[1]), fmaxf(w4[2], w4[3]));
+            for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
+            tmem_wait_ld();
+            const int j0 = j * BN;
+            const bool wtile = j >= jw0;
+            float mxg = -INFINITY, mxl = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 128; ++c) {
+                const float sv = __uint_as_float(r[c >> 5][c & 31]);
+                const bool sel = ((mwords[c >> 5] >> (c & 31)) & 1u) && (j0 + c <= pos);
+                if (sel) mxg = fmaxf(mxg, sv);
+                if (wtile && j0 + c >= lo_w && j0 + c <= pos) mxl = fmaxf(mxl, sv);
             }
-            float *x = &sh_xch[buf][0][0];
-            x[(2 * half + 0) * 128 + tw] = mxg;
-            x[(2 * half + 1) * 128 + tw] = mxl;
-            named_bar(bar_id, 64);
-            if (*abort) break;                                      // both warps of the pair agree here
-            mxg = fmaxf(mxg, x[(2 * (1 - half) + 0) * 128 + tw]);
-            mxl = fmaxf(mxl, x[(2 * (1 - half) + 1) * 128 + tw]);
             // PV of the previous tile must be done before O is touched
             if (j > 0) {
-                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->o_done), (j - 1) & 1, p.wait_ns, abort)))
-                    continue;                                       // next barrier sees the abort
+                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->o_done), (j - 1) & 1, p.wait_ns, abort));
+                if (!ok) break;
                 tc_fence_after();
             }
             const float mxg2 = mxg * c2, mxl2 = mxl * c2;
             if (__any_sync(0xffffffffu, mxg2 > mg + 8.0f)) {
                 const float mn = fmaxf(mg, mxg2);
                 if (j > 0) {
-                    const float corr = (mn == -INFINITY) ? 1.f : (mg == -INFINITY ? 0.f : ex2(mg - mn));
+                    const float corr = (mn == -INFINITY || mg == -INFINITY) ? (mn == -INFINITY ? 1.f : 0.f) : ex2(mg - mn);
                     lg *= corr;
-                    tmem_scale64(tOg, corr);
+                    cg *= corr;
+                    tmem_scale128(tOg, corr);
                 }
                 mg = mn;
             }
             if (wtile && __any_sync(0xffffffffu, mxl2 > ml + 8.0f)) {
                 const float mn = fmaxf(ml, mxl2);
                 if (j > jw0) {
-                    const float corr = (mn == -INFINITY) ? 1.f : (ml == -INFINITY ? 0.f : ex2(ml - mn));
+                    const float corr = (mn == -INFINITY || ml == -INFINITY) ? (mn == -INFINITY ? 1.f : 0.f) : ex2(ml - mn);
                     ll *= corr;
-                    tmem_scale64(tOl, corr);
+                    cl *= corr;
+                    tmem_scale128(tOl, corr);
                 }
                 ml = mn;
             }
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
-            {
+            float sg0 = 0.f, sg1 = 0.f, sl0 = 0.f, sl1 = 0.f;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const int c = 2 * e;
-                    bool q0 = ((c < 32 ? mw0 : mw1) >> (c & 31)) & 1u;
-                    bool q1 = ((c + 1 < 32 ? mw0 : mw1) >> ((c + 1) & 31)) & 1u;
-                    if (diag) {
-                        q0 = q0 && (j0 + c <= pos);
-                        q1 = q1 && (j0 + c + 1 <= pos);
-                    }
-                    const float a = q0 ? ex2(fmaf(s[c], c2, -mg)) : 0.f;
-                    const float bb = q1 ? ex2(fmaf(s[c + 1], c2, -mg)) : 0.f;
-                    a4[e & 1] += a;
-                    a4[2 + (e & 1)] += bb;
+                    const int c = hf * 64 + 2 * e;
+                    const float s0 = __uint_as_float(r[c >> 5][c & 31]);
+                    const float s1 = __uint_as_float(r[(c + 1) >> 5][(c + 1) & 31]);
+                    const bool q0 = ((mwords[c >> 5] >> (c & 31)) & 1u) && (j0 + c <= pos);
+                    const bool q1 = ((mwords[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u) && (j0 + c + 1 <= pos);
+                    const float a = q0 ? ex2(fmaf(s0, c2, -mg)) : 0.f;
+                    const float bb = q1 ? ex2(fmaf(s1, c2, -mg)) : 0.f;
+                    sg0 += a;
+                    sg1 += bb;
                     pk[e] = pack_bf16(a, bb);
                 }
-                tmem_st32(tS + 32 * half, pk);
+                tmem_st32(tS + 32 * hf, pk);
             }
-            lg += (a4[0] + a4[1]) + (a4[2] + a4[3]);
             if (wtile) {
-                float b4[4] = {0.f, 0.f, 0.f, 0.f};
-                uint32_t pk[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int c = 2 * e;
-                    const bool w0 = j0 + c >= lo_w && j0 + c <= pos;
-                    const bool w1 = j0 + c + 1 >= lo_w && j0 + c + 1 <= pos;
-                    const float a = w0 ? ex2(fmaf(s[c], c2, -ml)) : 0.f;
-                    const float bb = w1 ? ex2(fmaf(s[c + 1], c2, -ml)) : 0.f;
-                    b4[e & 1] += a;
-                    b4[2 + (e & 1)] += bb;
-                    pk[e] = pack_bf16(a, bb);
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int c = hf * 64 + 2 * e;
+                        const float s0 = __uint_as_float(r[c >> 5][c & 31]);
+                        const float s1 = __uint_as_float(r[(c + 1) >> 5][(c + 1) & 31]);
+                        const bool w0 = j0 + c >= lo_w && j0 + c <= pos;
+                        const bool w1 = j0 + c + 1 >= lo_w && j0 + c + 1 <= pos;
+                        const float a = w0 ? ex2(fmaf(s0, c2, -ml)) : 0.f;
+                        const float bb = w1 ? ex2(fmaf(s1, c2, -ml)) : 0.f;
+                        sl0 += a;
+                        sl1 += bb;
+                        pk[e] = pack_bf16(a, bb);
+                    }
+                    tmem_st32(tS + 64 + 32 * hf, pk);
                 }
-                tmem_st32(tS + 64 + 32 * half, pk);
-                ll += (b4[0] + b4[1]) + (b4[2] + b4[3]);
             }
             tmem_wait_st();
+            {
+                const float y = (sg0 + sg1) - cg;
+                const float t = lg + y;
+                cg = (t - lg) - y;
+                lg = t;
+            }
+            {
+                const float y = (sl0 + sl1) - cl;
+                const float t = ll + y;
+                cl = (t - ll) - y;
+                ll = t;
+            }
             tc_fence_before();
             mbar_arrive(smem_u32(&bars->p_full));
         }
-        // combine the two halves' row sums (every softmax warp reaches this barrier)
-        {
-            float *x = &sh_xch[0][0][0];
-            named_bar(bar_id, 64);
-            x[(2 * half + 0) * 128 + tw] = lg;
-            x[(2 * half + 1) * 128 + tw] = ll;
-            named_bar(bar_id, 64);
-            lg += x[(2 * (1 - half) + 0) * 128 + tw];
-            ll += x[(2 * (1 - half) + 1) * 128 + tw];
-        }
-        const bool fin = __all_sync(0xffffffffu, !*abort && mbar_wait(smem_u32(&bars->o_final), 0, p.wait_ns, abort));
+        const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(smem_u32(&bars->o_final), 0, p.wait_ns, abort));
         if (fin) {
             tc_fence_after();
             const float ig = lg > 0.f ? 1.f / lg : 0.f;
             const float il = ll > 0.f ? 1.f / ll : 0.f;
             float sgate = 0.f;
             if (valid) {
-                const float xg = p.gate[((size_t)b * p.Lq + row) * p.Hq + h];
-                sgate = 1.0f / (1.0f + expf(-xg));
+                const float x = p.gate[((size_t)b * p.Lq + row) * p.Hq + h];
+                sgate = 1.0f / (1.0f + expf(-x));
             }
-            const size_t orow = (((size_t)b * p.Lq + row) * p.Hq + h) * HD + 64 * half;
+            const size_t orow = (((size_t)b * p.Lq + row) * p.Hq + h) * HD;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 uint32_t og[32], ol[32];
                 tmem_ld32(tOg + 32 * c, og);
                 tmem_ld32(tOl + 32 * c, ol);

@@ -13,11 +13,9 @@
 //
 // Rows whose causal length fits (kSmemKeys) are first copied into shared
 // memory, so only that one read touches L2/HBM; longer rows are re-read from
-// global memory each pass.  Histogram updates are aggregated per warp
-// (__match_any_sync): near-flat score rows put almost every key in one bin,
-// and unaggregated shared atomics on one address serialise.  The compaction
-// uses per-warp ballot counts and one scan over warps instead of block-wide
-// scans per element chunk.
+// global memory each pass.  The bin holding the k-th key is found by a
+// block-parallel scan over the bins (descending); the compaction uses
+// per-warp ballot counts and one pass over warp totals.
 #include "common.cuh"
 #include "internal.h"
 
@@ -32,13 +30,55 @@ constexpr int kHistBins = 2048;
 struct TopkShared {
     unsigned int hist[kHistBins];
     unsigned int sh_digit, sh_remaining;
+    unsigned int wsum[NW], woff[NW];
     int cnt_gt[NW], cnt_eq[NW];
 };
 
-__device__ __forceinline__ void hist_add(unsigned int *hist, bool take, unsigned int bin, int lane) {
-    const unsigned int key = take ? bin : (0x80000000u | (unsigned)lane);   // unmatched lanes stay alone
-    const unsigned int peers = __match_any_sync(0xffffffffu, key);
-    if (take && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (unsigned)__popc(peers));
+// Find the bin (scanning from the top) in which the running count of keys
+// first reaches `remaining`; every thread owns nb / NT consecutive bins.
+// Writes the bin and the count still needed inside it to shared memory.
+__device__ __forceinline__ void find_bin(TopkShared &sh, unsigned int nb, unsigned int remaining, int tid) {
+    const int lane = tid & 31, warp = tid >> 5;
+    const int per = (int)nb / NT;
+    unsigned int c[kHistBins / NT];
+    unsigned int tot = 0;
+#pragma unroll
+    for (int k = 0; k < kHistBins / NT; ++k) {
+        c[k] = k < per ? sh.hist[nb - 1 - (unsigned)(per * tid + k)] : 0u;
+        tot += c[k];
+    }
+    unsigned int incl = tot;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const unsigned int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    if (lane == 31) sh.wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        unsigned int v = lane < NW ? sh.wsum[lane] : 0u;
+        unsigned int vi = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const unsigned int y = __shfl_up_sync(0xffffffffu, vi, off);
+            if (lane >= off) vi += y;
+        }
+        if (lane < NW) sh.woff[lane] = vi - v;
+    }
+    __syncthreads();
+    const unsigned int excl = sh.woff[warp] + incl - tot;
+    if (excl < remaining && remaining <= excl + tot) {
+        unsigned int cum = excl;
+#pragma unroll
+        for (int k = 0; k < kHistBins / NT; ++k) {
+            if (k < per && cum + c[k] >= remaining) {
+                sh.sh_digit = nb - 1 - (unsigned)(per * tid + k);
+                sh.sh_remaining = remaining - cum;
+                break;
+            }
+            cum += c[k];
+        }
+    }
 }
 
 template <bool SMEM>
@@ -66,49 +106,20 @@ topk_radix_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lk
         __syncthreads();
         u = row_cache;
     }
-    const int n_pad = (n + 31) & ~31;
 
     unsigned int prefix = 0, mask = 0, remaining = (unsigned int)topk;
-    const int shifts[3] = {20, 10, 0};
-    const int widths[3] = {11, 10, 10};
-#pragma unroll 1
+#pragma unroll
     for (int ps = 0; ps < 3; ++ps) {
-        const int shift = shifts[ps];
-        const unsigned int nb = 1u << widths[ps];
+        const int shift = ps == 0 ? 20 : (ps == 1 ? 10 : 0);
+        const unsigned int nb = ps == 0 ? 2048u : 1024u;
         for (int t = tid; t < (int)nb; t += NT) sh.hist[t] = 0;
         __syncthreads();
-        for (int j = tid; j < n_pad; j += NT) {
-            const bool in = j < n;
-            const unsigned int x = in ? (SMEM ? u[j] : __ldg(u + j)) : 0u;
-            const bool take = in && (x & mask) == prefix;
-            hist_add(sh.hist, take, (x >> shift) & (nb - 1u), lane);
+        for (int j = tid; j < n; j += NT) {
+            const unsigned int x = SMEM ? u[j] : __ldg(u + j);
+            if ((x & mask) == prefix) atomicAdd(&sh.hist[(x >> shift) & (nb - 1u)], 1u);
         }
         __syncthreads();
-        if (warp == 0) {
-            // lane covers bins nb-1-L*per .. nb-L*per-per (descending)
-            const int per = (int)nb / 32;
-            unsigned int tot = 0;
-            for (int t = 0; t < per; ++t) tot += sh.hist[nb - 1 - (lane * per + t)];
-            unsigned int incl = tot;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const unsigned int y = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += y;
-            }
-            const unsigned int excl = incl - tot;
-            if (excl < remaining && remaining <= incl) {
-                unsigned int cum = excl;
-                for (int t = 0; t < per; ++t) {
-                    const unsigned int c = sh.hist[nb - 1 - (lane * per + t)];
-                    if (cum + c >= remaining) {
-                        sh.sh_digit = nb - 1 - (unsigned)(lane * per + t);
-                        sh.sh_remaining = remaining - cum;
-                        break;
-                    }
-                    cum += c;
-                }
-            }
-        }
+        find_bin(sh, nb, remaining, tid);
         __syncthreads();
         prefix |= sh.sh_digit << shift;
         mask |= (nb - 1u) << shift;
