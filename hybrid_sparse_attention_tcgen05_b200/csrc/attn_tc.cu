@@ -218,9 +218,10 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                 for (int c = 0; c < 128; ++c)
                     if (j * BN + c > pos) s[c] = -INFINITY;
             }
-            float mx = s[0];
+            float m4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+            for (int c = 4; c < 128; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
+            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             const float mx2 = mx * c2;
             if (__any_sync(0xffffffffu, mx2 > m + 8.0f)) {
                 const float m_new = fmaxf(m, mx2);
@@ -228,14 +229,14 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                     const float corr = ex2(m - m_new);
                     l *= corr;
                     lc *= corr;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + 32 * c, o);
+#pragma unroll 1
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t o[16];
+                        tmem_ld16(tO + 16 * c, o);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
-                        tmem_st32(tO + 32 * c, o);
+                        for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+                        tmem_st16(tO + 16 * c, o);
                     }
                     tmem_wait_st();
                 }
@@ -243,17 +244,17 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             }
             float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t pk[32];
+            for (int qq = 0; qq < 4; ++qq) {
+                uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int c = hf * 64 + 2 * e;
+                for (int e = 0; e < 16; ++e) {
+                    const int c = qq * 32 + 2 * e;
                     const float a = ex2(fmaf(s[c], c2, -m));
                     const float bb = ex2(fmaf(s[c + 1], c2, -m));
                     if (e & 1) { ps2 += a; ps3 += bb; } else { ps0 += a; ps1 += bb; }
                     pk[e] = pack_bf16(a, bb);
                 }
-                tmem_st32(tS + 32 * hf, pk);
+                tmem_st16(tS + 16 * qq, pk);
             }
             tmem_wait_st();
             const float ts = (ps0 + ps1) + (ps2 + ps3);
@@ -308,7 +309,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 constexpr int SC_Q_STAGES = 3;
 constexpr int SC_K_STAGES = 2;
 constexpr int SC_BUFS = 4;
-constexpr int SC_THREADS = 192;   // warps 0-3 scores, 4 TMA, 5 MMA
+constexpr int SC_THREADS = 320;   // warps 0-7 scores (two per lane quarter), 8 TMA, 9 MMA
 
 struct ScBars {
     uint64_t q_full[SC_Q_STAGES], q_empty[SC_Q_STAGES];
@@ -363,7 +364,7 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         }
         for (int s = 0; s < SC_BUFS; ++s) {
             mbar_init(smem_u32(&bars->s_full[s]), 1);
-            mbar_init(smem_u32(&bars->s_free[s]), 128);
+            mbar_init(smem_u32(&bars->s_free[s]), 256);
         }
         mbar_init(smem_u32(&bars->drain), 1);
         bars->abort = 0;
@@ -379,7 +380,7 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     const uint32_t tmem = bars->tmem_base;
     volatile int *abort = &bars->abort;
 
-    if (warp == 4) {
+    if (warp == 8) {
         if (lane == 0) {
             tma_prefetch(&tq);
             tma_prefetch(&tk);
@@ -410,7 +411,7 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     mbar_drain(smem_u32(&bars->q_full[it % SC_Q_STAGES]), (it / SC_Q_STAGES) & 1);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         if (lane == 0) {
             bool ok = true;
             for (int j = 0; ok && j < n_kv; ++j) {
@@ -433,20 +434,23 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         }
     } else {
         // ------------------------------------------------ score warps
-        const int tw = threadIdx.x;
+        // warp w serves TMEM lanes 32*(w%4).. and columns 64*(w/4) .. +63
+        const int q4 = warp & 3, half = warp >> 2;
+        const int tw = 32 * q4 + lane;
         const int row = r0 + tw;
         const bool valid = row < r_end;
         const int pos = off + min(row, r_end - 1);
-        const uint32_t lane_off = (uint32_t)(tw & ~31) << 16;
+        const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
+        const uint32_t colh = (uint32_t)(64 * half);
         const float c2 = p.scale_log2;
         float *srow = valid ? p.scores + (((size_t)b * p.Hkv + g) * p.row_count + (row - p.row_begin)) * p.ld
                             : nullptr;
         const bool vec4 = (p.ld & 3) == 0;
         bool ok = true;
         for (int j = 0; ok && j < n_kv; ++j) {
-            float acc[128];
+            float acc[64];
 #pragma unroll
-            for (int c = 0; c < 128; ++c) acc[c] = 0.f;
+            for (int c = 0; c < 64; ++c) acc[c] = 0.f;
             for (int hh = 0; hh < G; ++hh) {
                 const int it = j * G + hh, buf = it % SC_BUFS;
                 const float2 st = valid ? p.stats[((size_t)b * p.Hq + g * G + hh) * p.Lq + row]
@@ -454,36 +458,36 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[buf]), (it / SC_BUFS) & 1, p.wait_ns, abort));
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t tS = tmem + lane_off + (uint32_t)(buf * 128);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tS + 32 * c, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        acc[32 * c + e] = fmaf(ex2(fmaf(__uint_as_float(r[e]), c2, -st.x)), st.y, acc[32 * c + e]);
-                }
+                const uint32_t tS = tmem + lane_off + (uint32_t)(buf * 128) + colh;
+                uint32_t r[2][32];
+                tmem_ld32(tS, r[0]);
+                tmem_ld32(tS + 32, r[1]);
+                tmem_wait_ld();
                 tc_fence_before();
-                mbar_arrive(smem_u32(&bars->s_free[buf]));
+                mbar_arrive(smem_u32(&bars->s_free[buf]));   // S is in registers; the MMA may reuse the buffer
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    acc[c] = fmaf(ex2(fmaf(__uint_as_float(r[c >> 5][c & 31]), c2, -st.x)), st.y, acc[c]);
             }
             if (!ok) break;
             if (valid) {
-                const int j0 = j * BN;
-                const int lim = min(BN, p.Lkv - j0);      // columns inside the cache
+                const int j0 = j * BN + 64 * half;
+                const int lim = min(64, p.Lkv - j0);      // columns inside the cache
                 const int keep = min(lim, pos - j0 + 1);  // causal columns
                 float *dst = srow + j0;
-                if (vec4 && lim == BN) {
+                if (lim > 0) {
+                    if (vec4 && lim == 64) {
 #pragma unroll
-                    for (int c = 0; c < 128; c += 4) {
-                        float4 v4 = make_float4(c < keep ? acc[c] : 0.f, c + 1 < keep ? acc[c + 1] : 0.f,
-                                                c + 2 < keep ? acc[c + 2] : 0.f, c + 3 < keep ? acc[c + 3] : 0.f);
-                        *reinterpret_cast<float4 *>(dst + c) = v4;
+                        for (int c = 0; c < 64; c += 4) {
+                            float4 v4 = make_float4(c < keep ? acc[c] : 0.f, c + 1 < keep ? acc[c + 1] : 0.f,
+                                                    c + 2 < keep ? acc[c + 2] : 0.f, c + 3 < keep ? acc[c + 3] : 0.f);
+                            *reinterpret_cast<float4 *>(dst + c) = v4;
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 64; ++c)
+                            if (c < lim) dst[c] = c < keep ? acc[c] : 0.f;
                     }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 128; ++c)
-                        if (c < lim) dst[c] = c < keep ? acc[c] : 0.f;
                 }
             }
         }

@@ -60,14 +60,14 @@ struct SdParams {
 
 // Rescale 128 columns of an accumulator row in TMEM by `corr` (per thread).
 __device__ __forceinline__ void tmem_scale128(uint32_t t, float corr) {
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        tmem_ld32(t + 32 * c, o);
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+        uint32_t o[16];
+        tmem_ld16(t + 16 * c, o);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
-        tmem_st32(t + 32 * c, o);
+        for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+        tmem_st16(t + 16 * c, o);
     }
     tmem_wait_st();
 }
@@ -205,27 +205,77 @@ sparse_dense_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[buf]), (j >> 1) & 1, p.wait_ns, abort));
             if (!ok) break;
             tc_fence_after();
-            uint32_t r[4][32];
+            float sv[128];
+            {
+                uint32_t r[4][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
-            tmem_wait_ld();
+                for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(r[c >> 5][c & 31]);
+            }
             const int j0 = j * BN;
             const bool wtile = j >= jw0;
-            float mxg = -INFINITY, mxl = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                const float sv = __uint_as_float(r[c >> 5][c & 31]);
-                const bool sel = ((mwords[c >> 5] >> (c & 31)) & 1u) && (j0 + c <= pos);
-                if (sel) mxg = fmaxf(mxg, sv);
-                if (wtile && j0 + c >= lo_w && j0 + c <= pos) mxl = fmaxf(mxl, sv);
-            }
+            const bool diag = j0 + BN - 1 > pos_first;      // causal edge may cut this tile
             // PV of the previous tile must be done before O is touched
             if (j > 0) {
                 ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->o_done), (j - 1) & 1, p.wait_ns, abort));
                 if (!ok) break;
                 tc_fence_after();
             }
-            const float mxg2 = mxg * c2, mxl2 = mxl * c2;
+            float sl0 = 0.f, sl1 = 0.f;
+            if (wtile) {
+                // window branch first, on the unmasked scores
+                float w4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (j0 + c >= lo_w && j0 + c <= pos) w4[c & 3] = fmaxf(w4[c & 3], sv[c]);
+                const float mxl2 = fmaxf(fmaxf(w4[0], w4[1]), fmaxf(w4[2], w4[3])) * c2;
+                if (__any_sync(0xffffffffu, mxl2 > ml + 8.0f)) {
+                    const float mn = fmaxf(ml, mxl2);
+                    if (j > jw0) {
+                        const float corr = (mn == -INFINITY || ml == -INFINITY) ? (mn == -INFINITY ? 1.f : 0.f) : ex2(ml - mn);
+                        ll *= corr;
+                        cl *= corr;
+                        tmem_scale128(tOl, corr);
+                    }
+                    ml = mn;
+                }
+                const float mlx = ml == -INFINITY ? 0.f : ml;
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int c = qq * 32 + 2 * e;
+                        const bool w0 = j0 + c >= lo_w && j0 + c <= pos;
+                        const bool w1 = j0 + c + 1 >= lo_w && j0 + c + 1 <= pos;
+                        const float a = w0 ? ex2(fmaf(sv[c], c2, -mlx)) : 0.f;
+                        const float bb = w1 ? ex2(fmaf(sv[c + 1], c2, -mlx)) : 0.f;
+                        sl0 += a;
+                        sl1 += bb;
+                        pk[e] = pack_bf16(a, bb);
+                    }
+                    tmem_st16(tS + 64 + 16 * qq, pk);
+                }
+            }
+            // global branch: unselected keys become -inf in place (one select per key)
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (diag) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                    const bool sel = ((mwords[c >> 5] >> (c & 31)) & 1u) && (j0 + c <= pos);
+                    sv[c] = sel ? sv[c] : -INFINITY;
+                    m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                    sv[c] = ((mwords[c >> 5] >> (c & 31)) & 1u) ? sv[c] : -INFINITY;
+                    m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
+                }
+            }
+            const float mxg2 = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c2;
             if (__any_sync(0xffffffffu, mxg2 > mg + 8.0f)) {
                 const float mn = fmaxf(mg, mxg2);
                 if (j > 0) {
@@ -236,55 +286,24 @@ sparse_dense_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 }
                 mg = mn;
             }
-            if (wtile && __any_sync(0xffffffffu, mxl2 > ml + 8.0f)) {
-                const float mn = fmaxf(ml, mxl2);
-                if (j > jw0) {
-                    const float corr = (mn == -INFINITY || ml == -INFINITY) ? (mn == -INFINITY ? 1.f : 0.f) : ex2(ml - mn);
-                    ll *= corr;
-                    cl *= corr;
-                    tmem_scale128(tOl, corr);
-                }
-                ml = mn;
-            }
-            float sg0 = 0.f, sg1 = 0.f, sl0 = 0.f, sl1 = 0.f;
+            // global P: masked keys are -inf, so 2^(-inf) = 0 needs no select
+            const float mgx = mg == -INFINITY ? 0.f : mg;
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t pk[32];
+            for (int qq = 0; qq < 4; ++qq) {
+                uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int c = hf * 64 + 2 * e;
-                    const float s0 = __uint_as_float(r[c >> 5][c & 31]);
-                    const float s1 = __uint_as_float(r[(c + 1) >> 5][(c + 1) & 31]);
-                    const bool q0 = ((mwords[c >> 5] >> (c & 31)) & 1u) && (j0 + c <= pos);
-                    const bool q1 = ((mwords[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u) && (j0 + c + 1 <= pos);
-                    const float a = q0 ? ex2(fmaf(s0, c2, -mg)) : 0.f;
-                    const float bb = q1 ? ex2(fmaf(s1, c2, -mg)) : 0.f;
-                    sg0 += a;
-                    sg1 += bb;
+                for (int e = 0; e < 16; ++e) {
+                    const int c = qq * 32 + 2 * e;
+                    const float a = ex2(fmaf(sv[c], c2, -mgx));
+                    const float bb = ex2(fmaf(sv[c + 1], c2, -mgx));
+                    a4[e & 1] += a;
+                    a4[2 + (e & 1)] += bb;
                     pk[e] = pack_bf16(a, bb);
                 }
-                tmem_st32(tS + 32 * hf, pk);
+                tmem_st16(tS + 16 * qq, pk);
             }
-            if (wtile) {
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int c = hf * 64 + 2 * e;
-                        const float s0 = __uint_as_float(r[c >> 5][c & 31]);
-                        const float s1 = __uint_as_float(r[(c + 1) >> 5][(c + 1) & 31]);
-                        const bool w0 = j0 + c >= lo_w && j0 + c <= pos;
-                        const bool w1 = j0 + c + 1 >= lo_w && j0 + c + 1 <= pos;
-                        const float a = w0 ? ex2(fmaf(s0, c2, -ml)) : 0.f;
-                        const float bb = w1 ? ex2(fmaf(s1, c2, -ml)) : 0.f;
-                        sl0 += a;
-                        sl1 += bb;
-                        pk[e] = pack_bf16(a, bb);
-                    }
-                    tmem_st32(tS + 64 + 32 * hf, pk);
-                }
-            }
+            const float sg0 = a4[0] + a4[2], sg1 = a4[1] + a4[3];
             tmem_wait_st();
             {
                 const float y = (sg0 + sg1) - cg;
