@@ -117,7 +117,7 @@ int run_topk(const Shape &s, const float *scores, long long ld, int row_begin, i
 // measured) with the gather (k_eff + w_eff K and V rows of 256 bytes per row
 // and KV head at kGatherBytesPerS, measured).
 // HYSPARSE_SPARSE_PATH=dense|gather overrides it.
-constexpr double kDenseTileCycles = 10000.0;
+constexpr double kDenseTileCycles = 4000.0;
 constexpr double kGatherBytesPerS = 6.0e12;
 bool prefer_dense_sparse(const Shape &s, int topk, int window) {
     if (!sparse_dense_supported(s)) return false;
