@@ -31,6 +31,7 @@ EXPORTS = (
     "hysparse_block",
     "hysparse_full_attn_scores_noalloc",
     "hysparse_workspace_status",
+    "hysparse_selftest_exp2",
     "hysparse_status_string",
     "hysparse_version",
 )
@@ -75,6 +76,8 @@ def lib():
     L.hysparse_block.restype = I
     L.hysparse_full_attn_scores_noalloc.argtypes = [SP, P, P, P, P, P, P, LL, I, I, P]
     L.hysparse_full_attn_scores_noalloc.restype = I
+    L.hysparse_selftest_exp2.argtypes = [P, P, P, I, P]
+    L.hysparse_selftest_exp2.restype = I
     L.hysparse_workspace_status.argtypes = [P, P]
     L.hysparse_workspace_status.restype = I
     L.hysparse_status_string.argtypes = [I]

@@ -40,6 +40,14 @@ namespace hs {
 namespace tc {
 namespace {
 
+// Share of the softmax exponentials computed by exp2_poly on the FMA pipe
+// instead of the MUFU unit: every kFwdPolyEvery-th element of the forward
+// pass, every kScPolyEvery-th of the score pass (0 = none).  Measured on
+// B200 at 1/4..1/2 offload both passes got slower (they are issue- and
+// latency-bound, not MUFU-bound), so both are off.
+constexpr int kFwdPolyEvery = 0;
+constexpr int kScPolyEvery = 0;
+
 struct FwdBars {
     uint64_t q_full;
     uint64_t kv_full[KV_STAGES];
@@ -249,8 +257,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int c = qq * 32 + 2 * e;
-                    const float a = ex2(fmaf(s[c], c2, -m));
-                    const float bb = ex2(fmaf(s[c + 1], c2, -m));
+                    const float a = ex2_mix<kFwdPolyEvery>(fmaf(s[c], c2, -m), c);
+                    const float bb = ex2_mix<kFwdPolyEvery>(fmaf(s[c + 1], c2, -m), c + 1);
                     if (e & 1) { ps2 += a; ps3 += bb; } else { ps0 += a; ps1 += bb; }
                     pk[e] = pack_bf16(a, bb);
                 }
@@ -467,7 +475,8 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 mbar_arrive(smem_u32(&bars->s_free[buf]));   // S is in registers; the MMA may reuse the buffer
 #pragma unroll
                 for (int c = 0; c < 64; ++c)
-                    acc[c] = fmaf(ex2(fmaf(__uint_as_float(r[c >> 5][c & 31]), c2, -st.x)), st.y, acc[c]);
+                    acc[c] = fmaf(ex2_mix<kScPolyEvery>(fmaf(__uint_as_float(r[c >> 5][c & 31]), c2, -st.x), c),
+                                  st.y, acc[c]);
             }
             if (!ok) break;
             if (valid) {
@@ -541,4 +550,21 @@ cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void
     return cudaGetLastError();
 }
 
+namespace {
+__global__ void selftest_exp2_kernel(const float *x, float *yp, float *ym, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) {
+        yp[i] = tc::exp2_poly(x[i]);
+        ym[i] = tc::ex2(x[i]);
+    }
+}
+}  // namespace
+
 }  // namespace hs
+
+extern "C" int hysparse_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int n, hs_stream_t stream) {
+    if (n < 0 || (n > 0 && (x == nullptr || y_poly == nullptr || y_mufu == nullptr))) return HS_ERR_INVALID_ARG;
+    if (n == 0) return HS_OK;
+    hs::selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, (cudaStream_t)stream>>>(x, y_poly, y_mufu, n);
+    return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
+}

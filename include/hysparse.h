@@ -174,6 +174,12 @@ int hysparse_full_attn_scores_noalloc(const hs_shape *shape, const void *q, cons
  * it and returns it.  Returns HS_ERR_CUDA if the synchronisation fails. */
 int hysparse_workspace_status(void *ws, hs_stream_t stream);
 
+/* Diagnostic: y_poly[i] = the kernels' polynomial 2^x (FMA-pipe
+ * exponential used for part of the softmax elements) and y_mufu[i] = the
+ * hardware ex2 approximation, for n device floats x.  Lets a test check both
+ * against exact 2^x.  Errors: HS_ERR_INVALID_ARG, HS_ERR_CUDA. */
+int hysparse_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int n, hs_stream_t stream);
+
 /* Static text for a status code. */
 const char *hysparse_status_string(int status);
 
