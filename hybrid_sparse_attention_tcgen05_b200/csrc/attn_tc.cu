@@ -48,19 +48,23 @@ namespace {
 constexpr int kFwdPolyEvery = 0;
 constexpr int kScPolyEvery = 0;
 
+constexpr int FWD_KV = 3;   // K/V ring slots (shared memory also holds Q0, Q1, P0, P1)
+
 struct FwdBars {
     uint64_t q_full;
-    uint64_t kv_full[KV_STAGES];
-    uint64_t kv_empty[KV_STAGES];
-    uint64_t s_full[2];
-    uint64_t p_full[2];
-    uint64_t o_final[2];
+    uint64_t kv_full[FWD_KV];
+    uint64_t kv_empty[FWD_KV];
+    uint64_t s_full[2];    // S_w holds Q_w K_j^T           (MMA commit)
+    uint64_t s_free[2];    // softmax w has S_w in registers (128 arrivals)
+    uint64_t p_full[2];    // P_w written to shared memory   (128 arrivals)
+    uint64_t pv_done[2];   // O_w += P_w V_j completed; P_w buffer free (MMA commit)
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
 };
 
-constexpr size_t kFwdSmem = 1024 + 2 * TILE + KV_STAGES * TILE + sizeof(FwdBars);
+constexpr size_t kFwdSmem = 1024 + 2 * TILE + FWD_KV * TILE + 2 * TILE + sizeof(FwdBars);
+static_assert(kFwdSmem <= 232448, "forward kernel shared memory");
 
 struct FwdParams {
     int Lq, Lkv, Hq, Hkv, G;
@@ -73,6 +77,23 @@ struct FwdParams {
     unsigned long long wait_ns;
 };
 
+// O (+)= P V with P a 128x128 bf16 tile in shared memory (K-major, 128-byte
+// swizzle, the layout of a Q tile) and V an N-major tile.
+__device__ __forceinline__ void issue_pv_ss(uint32_t d_tmem, uint32_t p_addr, uint32_t v_addr, bool accumulate) {
+    constexpr uint32_t I = idesc_bf16(128, 128, false, true);
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; ++kk) {
+        const uint32_t o = (kk >> 2) * HALF + (kk & 3) * 32;
+        mma_ss(d_tmem, sdesc_sw128(p_addr + o, 16, 1024), sdesc_sw128(v_addr + kk * 2048, HALF, 1024), I,
+               (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+// KV ring order = MMA consumption order: K0, K1, V0, K2, V1, K3, V2, ...
+// (S_{j+1} = Q K_{j+1}^T is issued before O += P_j V_j).
+__device__ __forceinline__ int kv_seq_k(int j) { return j == 0 ? 0 : 2 * j - 1; }
+__device__ __forceinline__ int kv_seq_v(int j, int n) { return j + 1 < n ? 2 * j + 2 : 2 * j + 1; }
+
 __global__ void __launch_bounds__(FWD_THREADS, 1)
 attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
             const __grid_constant__ CUtensorMap tv, const FwdParams p) {
@@ -80,7 +101,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     uint8_t *smem = align1024(smem_raw);
     uint8_t *sq = smem;
     uint8_t *skv = smem + 2 * TILE;
-    FwdBars *bars = reinterpret_cast<FwdBars *>(smem + 2 * TILE + KV_STAGES * TILE);
+    uint8_t *sp = smem + 2 * TILE + FWD_KV * TILE;
+    FwdBars *bars = reinterpret_cast<FwdBars *>(smem + 4 * TILE + FWD_KV * TILE);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tile = gridDim.x - 1 - blockIdx.x;  // heaviest row tiles first
@@ -96,14 +118,15 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&bars->q_full), 1);
-        for (int s = 0; s < KV_STAGES; ++s) {
+        for (int s = 0; s < FWD_KV; ++s) {
             mbar_init(smem_u32(&bars->kv_full[s]), 1);
             mbar_init(smem_u32(&bars->kv_empty[s]), 1);
         }
         for (int w = 0; w < 2; ++w) {
             mbar_init(smem_u32(&bars->s_full[w]), 1);
+            mbar_init(smem_u32(&bars->s_free[w]), 128);
             mbar_init(smem_u32(&bars->p_full[w]), 128);
-            mbar_init(smem_u32(&bars->o_final[w]), 1);
+            mbar_init(smem_u32(&bars->pv_done[w]), 1);
         }
         mbar_init(smem_u32(&bars->drain), 1);
         bars->abort = 0;
@@ -132,66 +155,65 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                     tma_load_4d(smem_u32(sq + s * TILE + hf * HALF), &tq, qb, hf * 64, h0 + s, r0, b);
             int issued = 0;
             for (int it = 0; it < 2 * n_kv; ++it) {
-                const int slot = it % KV_STAGES, use = it / KV_STAGES;
+                // sequence position -> which tile: 0 -> K0, then (K_{m+1}, V_m) pairs, last V_{n-1}
+                int j, is_v;
+                if (it == 0) { j = 0; is_v = 0; }
+                else if (it == 2 * n_kv - 1) { j = n_kv - 1; is_v = 1; }
+                else { is_v = (it & 1) == 0; j = is_v ? (it - 2) / 2 : (it + 1) / 2; }
+                const int slot = it % FWD_KV, use = it / FWD_KV;
                 if (!mbar_wait(smem_u32(&bars->kv_empty[slot]), (use & 1) ^ 1, p.wait_ns, abort)) break;
                 const uint32_t fb = smem_u32(&bars->kv_full[slot]);
                 mbar_expect_tx(fb, TILE);
-                const CUtensorMap *m = (it & 1) ? &tv : &tk;
-                const int j = it >> 1;
+                const CUtensorMap *m = is_v ? &tv : &tk;
                 for (int hf = 0; hf < 2; ++hf)
                     tma_load_4d(smem_u32(skv + slot * TILE + hf * HALF), m, fb, hf * 64, g, j * BN, b);
                 issued = it + 1;
             }
             if (*abort) {  // let our own copies land before the CTA goes away
                 mbar_drain(qb, 0);
-                for (int it = issued > KV_STAGES ? issued - KV_STAGES : 0; it < issued; ++it)
-                    mbar_drain(smem_u32(&bars->kv_full[it % KV_STAGES]), (it / KV_STAGES) & 1);
+                for (int it = issued > FWD_KV ? issued - FWD_KV : 0; it < issued; ++it)
+                    mbar_drain(smem_u32(&bars->kv_full[it % FWD_KV]), (it / FWD_KV) & 1);
             }
         }
     } else if (warp == 9) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
-            const uint32_t q0 = smem_u32(sq), q1 = smem_u32(sq + TILE);
+            const uint32_t tS[2] = {tmem, tmem + 128}, tO[2] = {tmem + 256, tmem + 384};
+            const uint32_t qa[2] = {smem_u32(sq), smem_u32(sq + TILE)};
+            const uint32_t pa[2] = {smem_u32(sp), smem_u32(sp + TILE)};
             bool ok = mbar_wait(smem_u32(&bars->q_full), 0, p.wait_ns, abort);
-            // S for tile 0
             if (ok) ok = mbar_wait(smem_u32(&bars->kv_full[0]), 0, p.wait_ns, abort);
             if (ok) {
                 tc_fence_after();
-                const uint32_t ka = smem_u32(skv);
-                issue_qk(tS0, q0, ka);
-                mma_commit(smem_u32(&bars->s_full[0]));
-                issue_qk(tS1, q1, ka);
-                mma_commit(smem_u32(&bars->s_full[1]));
+                for (int w = 0; w < 2; ++w) {
+                    issue_qk(tS[w], qa[w], smem_u32(skv));
+                    mma_commit(smem_u32(&bars->s_full[w]));
+                }
                 mma_commit(smem_u32(&bars->kv_empty[0]));
             }
             for (int j = 0; ok && j < n_kv; ++j) {
-                const int itV = 2 * j + 1, slotV = itV % KV_STAGES;
-                const int itK = 2 * j + 2, slotK = itK % KV_STAGES;
-                const bool has_next = j + 1 < n_kv;
-                const uint32_t va = smem_u32(skv + slotV * TILE);
-                const uint32_t ka = smem_u32(skv + slotK * TILE);
-                if (!(ok = mbar_wait(smem_u32(&bars->kv_full[slotV]), (itV / KV_STAGES) & 1, p.wait_ns, abort))) break;
-                if (!(ok = mbar_wait(smem_u32(&bars->p_full[0]), j & 1, p.wait_ns, abort))) break;
-                tc_fence_after();
-                issue_pv(tO0, tS0, va, j > 0);
-                if (!has_next) mma_commit(smem_u32(&bars->o_final[0]));
-                if (has_next) {
-                    if (!(ok = mbar_wait(smem_u32(&bars->kv_full[slotK]), (itK / KV_STAGES) & 1, p.wait_ns, abort))) break;
+                if (j + 1 < n_kv) {
+                    const int itK = kv_seq_k(j + 1), sk = itK % FWD_KV;
+                    if (!(ok = mbar_wait(smem_u32(&bars->kv_full[sk]), (itK / FWD_KV) & 1, p.wait_ns, abort))) break;
+                    for (int w = 0; w < 2; ++w) {
+                        if (!(ok = mbar_wait(smem_u32(&bars->s_free[w]), j & 1, p.wait_ns, abort))) break;
+                        tc_fence_after();
+                        issue_qk(tS[w], qa[w], smem_u32(skv + sk * TILE));
+                        mma_commit(smem_u32(&bars->s_full[w]));
+                    }
+                    if (!ok) break;
+                    mma_commit(smem_u32(&bars->kv_empty[sk]));
+                }
+                const int itV = kv_seq_v(j, n_kv), sv = itV % FWD_KV;
+                if (!(ok = mbar_wait(smem_u32(&bars->kv_full[sv]), (itV / FWD_KV) & 1, p.wait_ns, abort))) break;
+                for (int w = 0; w < 2; ++w) {
+                    if (!(ok = mbar_wait(smem_u32(&bars->p_full[w]), j & 1, p.wait_ns, abort))) break;
                     tc_fence_after();
-                    issue_qk(tS0, q0, ka);
-                    mma_commit(smem_u32(&bars->s_full[0]));
+                    issue_pv_ss(tO[w], pa[w], smem_u32(skv + sv * TILE), j > 0);
+                    mma_commit(smem_u32(&bars->pv_done[w]));
                 }
-                if (!(ok = mbar_wait(smem_u32(&bars->p_full[1]), j & 1, p.wait_ns, abort))) break;
-                tc_fence_after();
-                issue_pv(tO1, tS1, va, j > 0);
-                mma_commit(smem_u32(&bars->kv_empty[slotV]));
-                if (!has_next) mma_commit(smem_u32(&bars->o_final[1]));
-                if (has_next) {
-                    issue_qk(tS1, q1, ka);
-                    mma_commit(smem_u32(&bars->s_full[1]));
-                    mma_commit(smem_u32(&bars->kv_empty[slotK]));
-                }
+                if (!ok) break;
+                mma_commit(smem_u32(&bars->kv_empty[sv]));
             }
             // all MMAs this thread issued have completed before TMEM is freed
             mma_commit(smem_u32(&bars->drain));
@@ -207,6 +229,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         const uint32_t lane_off = (uint32_t)(tw & ~31) << 16;
         const uint32_t tS = tmem + lane_off + (uint32_t)(w * 128);
         const uint32_t tO = tmem + lane_off + 256u + (uint32_t)(w * 128);
+        uint8_t *prow = sp + w * TILE + tw * 128;      // this row of P (two 16 KB halves)
+        const int sw = tw & 7;                          // 128-byte swizzle phase of the row
         const float c2 = p.scale_log2;
         float m = -INFINITY, l = 0.f, lc = 0.f;
         bool ok = true;
@@ -214,13 +238,17 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[w]), j & 1, p.wait_ns, abort));
             if (!ok) break;
             tc_fence_after();
-            uint32_t r[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
-            tmem_wait_ld();
             float s[128];
+            {
+                uint32_t r[4][32];
 #pragma unroll
-            for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(r[c >> 5][c & 31]);
+                for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(r[c >> 5][c & 31]);
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&bars->s_free[w]));       // the MMA may now write S_{j+1}
             if (j * BN + BN - 1 > pos_first) {
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
@@ -229,8 +257,13 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             float m4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
             for (int c = 4; c < 128; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
-            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            const float mx2 = mx * c2;
+            const float mx2 = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c2;
+            // PV of the previous tile done: O is stable and the P buffer is free
+            if (j > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->pv_done[w]), (j - 1) & 1, p.wait_ns, abort));
+                if (!ok) break;
+                tc_fence_after();
+            }
             if (__any_sync(0xffffffffu, mx2 > m + 8.0f)) {
                 const float m_new = fmaxf(m, mx2);
                 if (j > 0) {
@@ -252,28 +285,30 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             }
             float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                uint32_t pk[16];
+            for (int ch = 0; ch < 16; ++ch) {           // 16-byte chunks of 8 keys
+                uint32_t pk[4];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int c = qq * 32 + 2 * e;
+                for (int e = 0; e < 4; ++e) {
+                    const int c = ch * 8 + 2 * e;
                     const float a = ex2_mix<kFwdPolyEvery>(fmaf(s[c], c2, -m), c);
                     const float bb = ex2_mix<kFwdPolyEvery>(fmaf(s[c + 1], c2, -m), c + 1);
                     if (e & 1) { ps2 += a; ps3 += bb; } else { ps0 += a; ps1 += bb; }
                     pk[e] = pack_bf16(a, bb);
                 }
-                tmem_st16(tS + 16 * qq, pk);
+                const int half = ch >> 3, c8 = ch & 7;
+                *reinterpret_cast<uint4 *>(prow + half * HALF + ((c8 ^ sw) << 4)) =
+                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
-            tmem_wait_st();
+            fence_proxy_async_smem();
+            mbar_arrive(smem_u32(&bars->p_full[w]));
             const float ts = (ps0 + ps1) + (ps2 + ps3);
             const float y = ts - lc;
             const float t = l + y;
             lc = (t - l) - y;
             l = t;
-            tc_fence_before();
-            mbar_arrive(smem_u32(&bars->p_full[w]));
         }
-        const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(smem_u32(&bars->o_final[w]), 0, p.wait_ns, abort));
+        const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(smem_u32(&bars->pv_done[w]), (n_kv - 1) & 1,
+                                                                 p.wait_ns, abort));
         if (fin) {
             tc_fence_after();
             const int h = h0 + w;
