@@ -349,7 +349,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 
 // ------------------------------------------------------------------ scores
 
-constexpr int SC_Q_STAGES = 3;
+constexpr int SC_Q_STAGES = 5;   // Q slots: all G query tiles stay resident when G <= 5, else a ring
 constexpr int SC_K_STAGES = 2;
 constexpr int SC_BUFS = 4;
 constexpr int SC_THREADS = 320;   // warps 0-7 scores (two per lane quarter), 8 TMA, 9 MMA
@@ -392,6 +392,7 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     const int g = blockIdx.y;
     const int b = blockIdx.z;
     const int G = p.G;
+    const bool resident = G <= SC_Q_STAGES;
     const int off = p.Lkv - p.Lq;
     const int pos_last = off + r_end - 1;
     const int n_kv = pos_last / BN + 1;
@@ -429,6 +430,14 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             tma_prefetch(&tk);
             int k_issued = 0, q_issued = 0;
             bool ok = true;
+            if (resident) {
+                for (int hh = 0; hh < G; ++hh) {
+                    const uint32_t qb = smem_u32(&bars->q_full[hh]);
+                    mbar_expect_tx(qb, TILE);
+                    for (int hf = 0; hf < 2; ++hf)
+                        tma_load_4d(smem_u32(sq + hh * TILE + hf * HALF), &tq, qb, hf * 64, g * G + hh, r0, b);
+                }
+            }
             for (int j = 0; ok && j < n_kv; ++j) {
                 const int sk_ = j % SC_K_STAGES;
                 if (!(ok = mbar_wait(smem_u32(&bars->k_empty[sk_]), ((j / SC_K_STAGES) & 1) ^ 1, p.wait_ns, abort))) break;
@@ -437,7 +446,7 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 for (int hf = 0; hf < 2; ++hf)
                     tma_load_4d(smem_u32(sk + sk_ * TILE + hf * HALF), &tk, kb, hf * 64, g, j * BN, b);
                 k_issued = j + 1;
-                for (int hh = 0; hh < G; ++hh) {
+                for (int hh = 0; !resident && hh < G; ++hh) {
                     const int it = j * G + hh, sq_ = it % SC_Q_STAGES;
                     if (!(ok = mbar_wait(smem_u32(&bars->q_empty[sq_]), ((it / SC_Q_STAGES) & 1) ^ 1, p.wait_ns, abort))) break;
                     const uint32_t qb = smem_u32(&bars->q_full[sq_]);
@@ -450,6 +459,8 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             if (*abort) {
                 for (int j = k_issued > SC_K_STAGES ? k_issued - SC_K_STAGES : 0; j < k_issued; ++j)
                     mbar_drain(smem_u32(&bars->k_full[j % SC_K_STAGES]), (j / SC_K_STAGES) & 1);
+                if (resident)
+                    for (int hh = 0; hh < G; ++hh) mbar_drain(smem_u32(&bars->q_full[hh]), 0);
                 for (int it = q_issued > SC_Q_STAGES ? q_issued - SC_Q_STAGES : 0; it < q_issued; ++it)
                     mbar_drain(smem_u32(&bars->q_full[it % SC_Q_STAGES]), (it / SC_Q_STAGES) & 1);
             }
@@ -462,13 +473,17 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 if (!(ok = mbar_wait(smem_u32(&bars->k_full[sk_]), (j / SC_K_STAGES) & 1, p.wait_ns, abort))) break;
                 const uint32_t ka = smem_u32(sk + sk_ * TILE);
                 for (int hh = 0; hh < G; ++hh) {
-                    const int it = j * G + hh, sq_ = it % SC_Q_STAGES, buf = it % SC_BUFS;
-                    if (!(ok = mbar_wait(smem_u32(&bars->q_full[sq_]), (it / SC_Q_STAGES) & 1, p.wait_ns, abort))) break;
+                    const int it = j * G + hh, buf = it % SC_BUFS;
+                    const int sq_ = resident ? hh : it % SC_Q_STAGES;
+                    if (!resident || j == 0) {
+                        const uint32_t par = resident ? 0u : (uint32_t)((it / SC_Q_STAGES) & 1);
+                        if (!(ok = mbar_wait(smem_u32(&bars->q_full[sq_]), par, p.wait_ns, abort))) break;
+                    }
                     if (!(ok = mbar_wait(smem_u32(&bars->s_free[buf]), ((it / SC_BUFS) & 1) ^ 1, p.wait_ns, abort))) break;
                     tc_fence_after();
                     issue_qk(tmem + (uint32_t)(buf * 128), smem_u32(sq + sq_ * TILE), ka);
                     mma_commit(smem_u32(&bars->s_full[buf]));
-                    mma_commit(smem_u32(&bars->q_empty[sq_]));
+                    if (!resident) mma_commit(smem_u32(&bars->q_empty[sq_]));
                 }
                 if (ok) mma_commit(smem_u32(&bars->k_empty[sk_]));
             }
