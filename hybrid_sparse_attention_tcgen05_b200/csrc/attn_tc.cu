@@ -66,6 +66,13 @@ struct FwdBars {
 constexpr size_t kFwdSmem = 1024 + 2 * TILE + FWD_KV * TILE + 2 * TILE + sizeof(FwdBars);
 static_assert(kFwdSmem <= 232448, "forward kernel shared memory");
 
+// What the pipeline computes.  FULL: causal attention of the full layer (O,
+// LSE, statistics for the score pass).  WIN: the sparse layer's window
+// branch (keys pos-window+1 .. pos), normalised into an fp32 buffer.  SEL:
+// the sparse layer's global branch (keys in the row's top-k set), merged
+// with the window branch by the gate into the layer output.
+enum FwdMode { FWD_FULL = 0, FWD_WIN = 1, FWD_SEL = 2 };
+
 struct FwdParams {
     int Lq, Lkv, Hq, Hkv, G;
     int row_begin, row_end;
@@ -75,6 +82,12 @@ struct FwdParams {
     float2 *stats;
     unsigned int *status;
     unsigned long long wait_ns;
+    // sparse-layer modes
+    int window, W;                   // window length; words per selection-mask row
+    const uint32_t *selmask;         // [B][Hkv][Lq][W]
+    float *wl;                       // [B][Lq][Hq][128] window branch, normalised (fp32)
+    const float *gate;               // [B][Lq][Hq]
+    __nv_bfloat16 *out_g, *out_l;    // optional branch outputs
 };
 
 // O (+)= P V with P a 128x128 bf16 tile in shared memory (K-major, 128-byte
@@ -94,6 +107,7 @@ __device__ __forceinline__ void issue_pv_ss(uint32_t d_tmem, uint32_t p_addr, ui
 __device__ __forceinline__ int kv_seq_k(int j) { return j == 0 ? 0 : 2 * j - 1; }
 __device__ __forceinline__ int kv_seq_v(int j, int n) { return j + 1 < n ? 2 * j + 2 : 2 * j + 1; }
 
+template <int MODE>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
 attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
             const __grid_constant__ CUtensorMap tv, const FwdParams p) {
@@ -114,7 +128,10 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     const int off = p.Lkv - p.Lq;
     const int pos_first = off + r0;
     const int pos_last = off + r_end - 1;
-    const int n_kv = pos_last / BN + 1;
+    // key tiles j_begin .. j_begin + n_kv - 1 (the window mode skips tiles no
+    // row's window reaches); loop counters below are relative to j_begin
+    const int j_begin = MODE == FWD_WIN ? max(0, pos_first - p.window + 1) / BN : 0;
+    const int n_kv = pos_last / BN + 1 - j_begin;
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&bars->q_full), 1);
@@ -166,7 +183,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                 mbar_expect_tx(fb, TILE);
                 const CUtensorMap *m = is_v ? &tv : &tk;
                 for (int hf = 0; hf < 2; ++hf)
-                    tma_load_4d(smem_u32(skv + slot * TILE + hf * HALF), m, fb, hf * 64, g, j * BN, b);
+                    tma_load_4d(smem_u32(skv + slot * TILE + hf * HALF), m, fb, hf * 64, g, (j_begin + j) * BN, b);
                 issued = it + 1;
             }
             if (*abort) {  // let our own copies land before the CTA goes away
@@ -232,9 +249,19 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         uint8_t *prow = sp + w * TILE + tw * 128;      // this row of P (two 16 KB halves)
         const int sw = tw & 7;                          // 128-byte swizzle phase of the row
         const float c2 = p.scale_log2;
+        const int lo_w = max(0, pos - p.window + 1);     // window mode: first key of the row's window
+        const uint4 *mrow = nullptr;                      // select mode: the row's top-k bitmask
+        uint4 mw = make_uint4(0, 0, 0, 0);
+        if (MODE == FWD_SEL) {
+            mrow = reinterpret_cast<const uint4 *>(p.selmask + (((size_t)b * p.Hkv + g) * p.Lq + (pos - off)) * p.W);
+            mw = __ldg(mrow);
+        }
         float m = -INFINITY, l = 0.f, lc = 0.f;
         bool ok = true;
         for (int j = 0; j < n_kv; ++j) {
+            const int j0 = (j_begin + j) * BN;           // key index of column 0
+            uint32_t mwords[4] = {mw.x, mw.y, mw.z, mw.w};
+            if (MODE == FWD_SEL && j + 1 < n_kv) mw = __ldg(mrow + j + 1);
             ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[w]), j & 1, p.wait_ns, abort));
             if (!ok) break;
             tc_fence_after();
@@ -249,10 +276,24 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&bars->s_free[w]));       // the MMA may now write S_{j+1}
-            if (j * BN + BN - 1 > pos_first) {
+            if (MODE == FWD_SEL) {
+                if (j0 + BN - 1 > pos_first) {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (!((mwords[c >> 5] >> (c & 31)) & 1u) || j0 + c > pos) s[c] = -INFINITY;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (!((mwords[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
+                }
+            } else if (MODE == FWD_WIN) {
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
-                    if (j * BN + c > pos) s[c] = -INFINITY;
+                    if (j0 + c > pos || j0 + c < lo_w) s[c] = -INFINITY;
+            } else if (j0 + BN - 1 > pos_first) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (j0 + c > pos) s[c] = -INFINITY;
             }
             float m4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
@@ -267,7 +308,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             if (__any_sync(0xffffffffu, mx2 > m + 8.0f)) {
                 const float m_new = fmaxf(m, mx2);
                 if (j > 0) {
-                    const float corr = ex2(m - m_new);
+                    // a row with nothing visible yet has m = -inf and an all-zero O row
+                    const float corr = m_new == -INFINITY ? 1.f : ex2(m - m_new);
                     l *= corr;
                     lc *= corr;
 #pragma unroll 1
@@ -283,6 +325,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                 }
                 m = m_new;
             }
+            const float mref = m == -INFINITY ? 0.f : m;   // masked keys (-inf) give 2^-inf = 0
             float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
 #pragma unroll
             for (int ch = 0; ch < 16; ++ch) {           // 16-byte chunks of 8 keys
@@ -290,8 +333,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int c = ch * 8 + 2 * e;
-                    const float a = ex2_mix<kFwdPolyEvery>(fmaf(s[c], c2, -m), c);
-                    const float bb = ex2_mix<kFwdPolyEvery>(fmaf(s[c + 1], c2, -m), c + 1);
+                    const float a = ex2_mix<kFwdPolyEvery>(fmaf(s[c], c2, -mref), c);
+                    const float bb = ex2_mix<kFwdPolyEvery>(fmaf(s[c + 1], c2, -mref), c + 1);
                     if (e & 1) { ps2 += a; ps3 += bb; } else { ps0 += a; ps1 += bb; }
                     pk[e] = pack_bf16(a, bb);
                 }
@@ -309,7 +352,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         }
         const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(smem_u32(&bars->pv_done[w]), (n_kv - 1) & 1,
                                                                  p.wait_ns, abort));
-        if (fin) {
+        if (fin && MODE == FWD_FULL) {
             tc_fence_after();
             const int h = h0 + w;
             const float inv_l = 1.0f / l;
@@ -334,6 +377,69 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                 const size_t si = ((size_t)b * p.Hq + h) * p.Lq + row;
                 p.lse[si] = (m + log2f(l)) * kLn2;
                 if (p.stats) p.stats[si] = make_float2(m, inv_l);
+            }
+        }
+        if (fin && MODE == FWD_WIN) {
+            // normalised window branch, fp32, for the select pass to merge
+            tc_fence_after();
+            const int h = h0 + w;
+            const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+            float4 *wrow = reinterpret_cast<float4 *>(p.wl + (((size_t)b * p.Lq + row) * p.Hq + h) * HD);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + 32 * c, o);
+                tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        wrow[8 * c + e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
+                                                      __uint_as_float(o[4 * e + 2]) * inv_l, __uint_as_float(o[4 * e + 3]) * inv_l);
+                }
+            }
+        }
+        if (fin && MODE == FWD_SEL) {
+            // out = sigmoid(gate) * global + (1 - sigmoid(gate)) * window
+            tc_fence_after();
+            const int h = h0 + w;
+            const float inv_l = l > 0.f ? 1.0f / l : 0.f;   // an empty top-k set gives a zero branch
+            const size_t ro = ((size_t)b * p.Lq + row) * p.Hq + h;
+            float sg = 0.f;
+            if (valid) sg = 1.0f / (1.0f + expf(-p.gate[ro]));
+            const float4 *wrow = reinterpret_cast<const float4 *>(p.wl + ro * HD);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + 32 * c, o);
+                tmem_wait_ld();
+                if (valid) {
+                    uint32_t po[16], pg[16], pl[16];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float4 wv = wrow[8 * c + e];
+                        const float g0 = __uint_as_float(o[4 * e]) * inv_l, g1 = __uint_as_float(o[4 * e + 1]) * inv_l;
+                        const float g2 = __uint_as_float(o[4 * e + 2]) * inv_l, g3 = __uint_as_float(o[4 * e + 3]) * inv_l;
+                        po[2 * e] = pack_bf16(sg * g0 + (1.f - sg) * wv.x, sg * g1 + (1.f - sg) * wv.y);
+                        po[2 * e + 1] = pack_bf16(sg * g2 + (1.f - sg) * wv.z, sg * g3 + (1.f - sg) * wv.w);
+                        pg[2 * e] = pack_bf16(g0, g1);
+                        pg[2 * e + 1] = pack_bf16(g2, g3);
+                        pl[2 * e] = pack_bf16(wv.x, wv.y);
+                        pl[2 * e + 1] = pack_bf16(wv.z, wv.w);
+                    }
+                    uint4 *d0 = reinterpret_cast<uint4 *>(p.out + ro * HD + 32 * c);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) d0[e] = make_uint4(po[4 * e], po[4 * e + 1], po[4 * e + 2], po[4 * e + 3]);
+                    if (p.out_g) {
+                        uint4 *d1 = reinterpret_cast<uint4 *>(p.out_g + ro * HD + 32 * c);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) d1[e] = make_uint4(pg[4 * e], pg[4 * e + 1], pg[4 * e + 2], pg[4 * e + 3]);
+                    }
+                    if (p.out_l) {
+                        uint4 *d2 = reinterpret_cast<uint4 *>(p.out_l + ro * HD + 32 * c);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) d2[e] = make_uint4(pl[4 * e], pl[4 * e + 1], pl[4 * e + 2], pl[4 * e + 3]);
+                    }
+                }
             }
         }
     }
@@ -582,21 +688,61 @@ cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void
         return cudaErrorInvalidValue;
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdSmem);
+        cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc<FWD_FULL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdSmem);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(attn_scores_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScSmem);
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
     const int n_tiles = (row_count + BM - 1) / BM;
-    FwdParams fp{s.Lq, s.Lkv, s.Hq, s.Hkv, s.G(), row_begin, row_begin + row_count,
-                 s.scale * kLog2e, (__nv_bfloat16 *)out, lse, stats, status, wait_ns};
-    attn_fwd_tc<<<dim3(n_tiles, s.Hq / 2, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp);
+    FwdParams fp{};
+    fp.Lq = s.Lq; fp.Lkv = s.Lkv; fp.Hq = s.Hq; fp.Hkv = s.Hkv; fp.G = s.G();
+    fp.row_begin = row_begin; fp.row_end = row_begin + row_count;
+    fp.scale_log2 = s.scale * kLog2e;
+    fp.out = (__nv_bfloat16 *)out; fp.lse = lse; fp.stats = stats; fp.status = status; fp.wait_ns = wait_ns;
+    attn_fwd_tc<FWD_FULL><<<dim3(n_tiles, s.Hq / 2, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || scores == nullptr) return e;
     ScParams sp{s.Lq, s.Lkv, s.Hq, s.Hkv, s.G(), row_begin, row_begin + row_count, row_count,
                 s.scale * kLog2e, stats, scores, ld, status, wait_ns};
     attn_scores_tc<<<dim3(n_tiles, s.Hkv, s.B), SC_THREADS, kScSmem, st>>>(mq, mk, sp);
+    return cudaGetLastError();
+}
+
+bool sparse_pair_supported(const Shape &s) {
+    return s.dtype == HS_BF16 && s.d == 128 && (s.G() % 2) == 0 && s.Lq >= 64;
+}
+
+size_t sparse_pair_wl_bytes(const Shape &s) { return (size_t)s.B * s.Lq * s.Hq * 128 * sizeof(float); }
+
+cudaError_t sparse_pair_tc_launch(const Shape &s, const void *q, const void *k, const void *v, const float *gate,
+                                  int window, void *out, void *og, void *ol, const uint32_t *mask, int W,
+                                  float *wl, unsigned int *status, unsigned long long wait_ns, cudaStream_t st) {
+    using namespace tc;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, s.Hq, s.Lq, s.B) || !make_map(&mk, k, s.Hkv, s.Lkv, s.B) ||
+        !make_map(&mv, v, s.Hkv, s.Lkv, s.B))
+        return cudaErrorInvalidValue;
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc<FWD_WIN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdSmem);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(attn_fwd_tc<FWD_SEL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdSmem);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    FwdParams fp{};
+    fp.Lq = s.Lq; fp.Lkv = s.Lkv; fp.Hq = s.Hq; fp.Hkv = s.Hkv; fp.G = s.G();
+    fp.row_begin = 0; fp.row_end = s.Lq;
+    fp.scale_log2 = s.scale * kLog2e;
+    fp.out = (__nv_bfloat16 *)out; fp.status = status; fp.wait_ns = wait_ns;
+    fp.window = window; fp.W = W; fp.selmask = mask; fp.wl = wl; fp.gate = gate;
+    fp.out_g = (__nv_bfloat16 *)og; fp.out_l = (__nv_bfloat16 *)ol;
+    const int n_tiles = (s.Lq + BM - 1) / BM;
+    attn_fwd_tc<FWD_WIN><<<dim3(n_tiles, s.Hq / 2, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attn_fwd_tc<FWD_SEL><<<dim3(n_tiles, s.Hq / 2, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp);
     return cudaGetLastError();
 }
 

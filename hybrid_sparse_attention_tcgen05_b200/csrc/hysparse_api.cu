@@ -46,7 +46,7 @@ struct WsLayout {
     size_t status = 0;
     size_t stats = 0, stats_end = 0;          // full layer per-row statistics
     size_t dec = 0, full_end = 0;             // decode split-K partials + logit stash
-    size_t selmask = 0, sparse_end = 0;       // dense-masked sparse layer: selection bitmask
+    size_t selmask = 0, wl = 0, sparse_end = 0;  // dense-masked sparse layer: bitmask, window branch
     size_t block_scores = 0, block_lse = 0, block_idx = 0;
     size_t total = 0;
 };
@@ -64,6 +64,8 @@ WsLayout ws_layout(const Shape &s, int topk, int row_chunk) {
     L.full_end = off;
     L.selmask = off;
     if (sparse_dense_supported(s)) off = align_up(off + selmask_bytes(s), 256);
+    L.wl = off;
+    if (sparse_dense_supported(s) && sparse_pair_supported(s)) off = align_up(off + sparse_pair_wl_bytes(s), 256);
     L.sparse_end = off;
     const int chunk = (row_chunk <= 0 || row_chunk > s.Lq) ? s.Lq : row_chunk;
     L.block_scores = off;
@@ -117,7 +119,8 @@ int run_topk(const Shape &s, const float *scores, long long ld, int row_begin, i
 // measured) with the gather (k_eff + w_eff K and V rows of 256 bytes per row
 // and KV head at kGatherBytesPerS, measured).
 // HYSPARSE_SPARSE_PATH=dense|gather overrides it.
-constexpr double kDenseTileCycles = 4000.0;
+constexpr double kDenseTileCycles = 4000.0;      // single-head kernel (odd G)
+constexpr double kPairTileCycles = 1700.0;       // paired-head pipeline (even G), per head
 constexpr double kGatherBytesPerS = 6.0e12;
 bool prefer_dense_sparse(const Shape &s, int topk, int window) {
     if (!sparse_dense_supported(s)) return false;
@@ -131,7 +134,8 @@ bool prefer_dense_sparse(const Shape &s, int topk, int window) {
         const double last = off + fmin((double)s.Lq, 128.0 * (t + 1)) - 1.0;
         tiles += floor(last / 128.0) + 1.0;
     }
-    const double dense_s = tiles * s.Hq * s.B * kDenseTileCycles / (148.0 * 1.9e9);
+    const double dense_s = tiles * s.Hq * s.B * (sparse_pair_supported(s) ? kPairTileCycles : kDenseTileCycles) /
+                           (148.0 * 1.9e9);
     double keys = 0.0;                         // sum over rows of k_eff + w_eff
     for (int i = 0; i < s.Lq; i += 64) {
         const double n = off + i + 1.0;
@@ -146,7 +150,16 @@ int run_sparse(const Shape &s, const void *q, const void *k, const void *v, cons
                cudaStream_t st) {
     unsigned int *status = reinterpret_cast<unsigned int *>(ws);
     if (prefer_dense_sparse(s, topk, window)) {
-        uint32_t *mask = reinterpret_cast<uint32_t *>(reinterpret_cast<char *>(ws) + ws_layout(s, topk, 1).selmask);
+        const WsLayout L = ws_layout(s, topk, 1);
+        uint32_t *mask = reinterpret_cast<uint32_t *>(reinterpret_cast<char *>(ws) + L.selmask);
+        if (sparse_pair_supported(s)) {
+            float *wl = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + L.wl);
+            cudaError_t e = selmask_build_launch(s, idx, topk, mask, status, st);
+            if (e == cudaSuccess)
+                e = sparse_pair_tc_launch(s, q, k, v, gate, window, out, og, ol, mask, selmask_words(s), wl, status,
+                                          wait_limit_ns(), st);
+            return cuda_status(e);
+        }
         return cuda_status(sparse_dense_tc_launch(s, q, k, v, idx, topk, gate, window, out, og, ol, mask,
                                                   status, wait_limit_ns(), st));
     }

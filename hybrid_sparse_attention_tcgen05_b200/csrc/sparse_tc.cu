@@ -416,6 +416,24 @@ bool sparse_dense_supported(const Shape &s) {
     return s.dtype == HS_BF16 && s.d == 128 && s.Lq >= 64 && selmask_words(s) * 4 * tc::SM_WARPS <= 96 * 1024;
 }
 
+cudaError_t selmask_build_launch(const Shape &s, const int32_t *idx, int topk, uint32_t *mask, unsigned int *status,
+                                 cudaStream_t st) {
+    using namespace tc;
+    const int W = selmask_words(s);
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(build_selmask, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    const long long n_rows = (long long)s.B * s.Hkv * s.Lq;
+    const long long mb = (n_rows + SM_WARPS - 1) / SM_WARPS;
+    if (mb > 0x7fffffffLL) return cudaErrorInvalidValue;
+    build_selmask<<<(unsigned)mb, SM_WARPS * 32, (size_t)SM_WARPS * W * 4, st>>>(idx, topk, s.Lq, s.Lkv, W, n_rows,
+                                                                                mask, status);
+    return cudaGetLastError();
+}
+
 cudaError_t sparse_dense_tc_launch(const Shape &s, const void *q, const void *k, const void *v,
                                    const int32_t *idx, int topk, const float *gate, int window, void *out,
                                    void *og, void *ol, uint32_t *mask, unsigned int *status,
