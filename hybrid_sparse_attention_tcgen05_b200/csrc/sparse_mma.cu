@@ -7,7 +7,7 @@
 // 128-token sliding window, out = gate*global + (1-gate)*local with a sigmoid
 // gate) and section 3.1 (the sparse layers only read the full layer's cache).
 //
-// One warp owns one (batch, query row, KV head) item: the G query heads of
+// One warp owns one (KV head, batch, query row) item: the G query heads of
 // that group share the item's key list.  Keys are gathered 32 at a time with
 // cp.async 16-byte copies (each warp instruction moves two whole 256-byte K or
 // V rows, so every L2 sector fetched is used) into a 3-stage shared-memory
@@ -274,10 +274,12 @@ __global__ void __launch_bounds__(SW * 32, 1) sparse_attn_mma(const SpParams p) 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long item = (long long)blockIdx.x * SW + warp;
     if (item >= (long long)p.B * p.Lq * p.Hkv) return;   // whole warp leaves together
-    const int g = (int)(item % p.Hkv);
-    const long long bi = item / p.Hkv;
-    const int i = (int)(bi % p.Lq);
-    const int b = (int)(bi / p.Lq);
+    // KV head slowest, then batch, then row: neighbouring warps gather from
+    // the same KV head's cache (which stays in L2) and have similar row lengths
+    const int i = (int)(item % p.Lq);
+    const long long bg = item / p.Lq;
+    const int b = (int)(bg % p.B);
+    const int g = (int)(bg / p.B);
     const int G = p.G;
     const int pos = p.Lkv - p.Lq + i;
     uint8_t *wbase = smem + warp * SpSmem<NB>::WARP_BYTES;
