@@ -277,9 +277,9 @@ __global__ void __launch_bounds__(SW * 32, 1) sparse_attn_mma(const SpParams p) 
     // KV head slowest, then batch, then row: neighbouring warps gather from
     // the same KV head's cache (which stays in L2) and have similar row lengths
     const int i = (int)(item % p.Lq);
-    const long long bg = item / p.Lq;
-    const int b = (int)(bg % p.B);
-    const int g = (int)(bg / p.B);
+    const long long head_batch = item / p.Lq;
+    const int b = (int)(head_batch % p.B);
+    const int g = (int)(head_batch / p.B);
     const int G = p.G;
     const int pos = p.Lkv - p.Lq + i;
     uint8_t *wbase = smem + warp * SpSmem<NB>::WARP_BYTES;
