@@ -28,7 +28,7 @@ from . import _lib
 from ._lib import HysparseError, HsShape
 
 __all__ = ["shape_of", "workspace_size", "alloc_workspace", "full_attn_scores", "topk",
-           "sparse_attn", "block", "workspace_status", "version", "HysparseError", "HsShape"]
+           "sparse_attn", "block", "workspace_status", "version", "launch_count", "HysparseError", "HsShape"]
 
 
 def _dtype_code(t: torch.dtype) -> int:
@@ -197,6 +197,11 @@ def workspace_status(ws: torch.Tensor) -> int:
     """Synchronise, read and clear the workspace status word (0 = ok)."""
     dev = _need_cuda(ws)
     return int(_lib.lib().hysparse_workspace_status(_ptr(ws), _stream(dev)))
+
+
+def launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(_lib.lib().hysparse_launch_count())
 
 
 def version() -> str:

@@ -32,6 +32,7 @@ EXPORTS = (
     "hysparse_full_attn_scores_noalloc",
     "hysparse_workspace_status",
     "hysparse_selftest_exp2",
+    "hysparse_launch_count",
     "hysparse_status_string",
     "hysparse_version",
 )
@@ -78,6 +79,8 @@ def lib():
     L.hysparse_full_attn_scores_noalloc.restype = I
     L.hysparse_selftest_exp2.argtypes = [P, P, P, I, P]
     L.hysparse_selftest_exp2.restype = I
+    L.hysparse_launch_count.argtypes = []
+    L.hysparse_launch_count.restype = ctypes.c_ulonglong
     L.hysparse_workspace_status.argtypes = [P, P]
     L.hysparse_workspace_status.restype = I
     L.hysparse_status_string.argtypes = [I]

@@ -700,12 +700,12 @@ cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void
     fp.row_begin = row_begin; fp.row_end = row_begin + row_count;
     fp.scale_log2 = s.scale * kLog2e;
     fp.out = (__nv_bfloat16 *)out; fp.lse = lse; fp.stats = stats; fp.status = status; fp.wait_ns = wait_ns;
-    attn_fwd_tc<FWD_FULL><<<dim3(n_tiles, s.Hq / 2, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp);
+    attn_fwd_tc<FWD_FULL><<<dim3(n_tiles, s.Hq / 2, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp); count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || scores == nullptr) return e;
     ScParams sp{s.Lq, s.Lkv, s.Hq, s.Hkv, s.G(), row_begin, row_begin + row_count, row_count,
                 s.scale * kLog2e, stats, scores, ld, status, wait_ns};
-    attn_scores_tc<<<dim3(n_tiles, s.Hkv, s.B), SC_THREADS, kScSmem, st>>>(mq, mk, sp);
+    attn_scores_tc<<<dim3(n_tiles, s.Hkv, s.B), SC_THREADS, kScSmem, st>>>(mq, mk, sp); count_launch();
     return cudaGetLastError();
 }
 
@@ -739,10 +739,10 @@ cudaError_t sparse_pair_tc_launch(const Shape &s, const void *q, const void *k, 
     fp.window = window; fp.W = W; fp.selmask = mask; fp.wl = wl; fp.gate = gate;
     fp.out_g = (__nv_bfloat16 *)og; fp.out_l = (__nv_bfloat16 *)ol;
     const int n_tiles = (s.Lq + BM - 1) / BM;
-    attn_fwd_tc<FWD_WIN><<<dim3(n_tiles, s.Hq / 2, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp);
+    attn_fwd_tc<FWD_WIN><<<dim3(n_tiles, s.Hq / 2, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp); count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    attn_fwd_tc<FWD_SEL><<<dim3(n_tiles, s.Hq / 2, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp);
+    attn_fwd_tc<FWD_SEL><<<dim3(n_tiles, s.Hq / 2, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp); count_launch();
     return cudaGetLastError();
 }
 
@@ -761,6 +761,6 @@ __global__ void selftest_exp2_kernel(const float *x, float *yp, float *ym, int n
 extern "C" int hysparse_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int n, hs_stream_t stream) {
     if (n < 0 || (n > 0 && (x == nullptr || y_poly == nullptr || y_mufu == nullptr))) return HS_ERR_INVALID_ARG;
     if (n == 0) return HS_OK;
-    hs::selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, (cudaStream_t)stream>>>(x, y_poly, y_mufu, n);
+    hs::selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, (cudaStream_t)stream>>>(x, y_poly, y_mufu, n); hs::count_launch();
     return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }

@@ -6,6 +6,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -145,16 +146,18 @@ bool prefer_dense_sparse(const Shape &s, int topk, int window) {
     return dense_s < gather_s;
 }
 
+// mask_ready: the dense path's selection bitmask in `ws` was already built
+// from this very index set (hysparse_block builds it once for all its layers).
 int run_sparse(const Shape &s, const void *q, const void *k, const void *v, const int32_t *idx,
                int topk, const float *gate, int window, void *out, void *og, void *ol, void *ws,
-               cudaStream_t st) {
+               cudaStream_t st, bool mask_ready = false) {
     unsigned int *status = reinterpret_cast<unsigned int *>(ws);
     if (prefer_dense_sparse(s, topk, window)) {
         const WsLayout L = ws_layout(s, topk, 1);
         uint32_t *mask = reinterpret_cast<uint32_t *>(reinterpret_cast<char *>(ws) + L.selmask);
         if (sparse_pair_supported(s)) {
             float *wl = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + L.wl);
-            cudaError_t e = selmask_build_launch(s, idx, topk, mask, status, st);
+            cudaError_t e = mask_ready ? cudaSuccess : selmask_build_launch(s, idx, topk, mask, status, st);
             if (e == cudaSuccess)
                 e = sparse_pair_tc_launch(s, q, k, v, gate, window, out, og, ol, mask, selmask_words(s), wl, status,
                                           wait_limit_ns(), st);
@@ -171,6 +174,9 @@ int run_sparse(const Shape &s, const void *q, const void *k, const void *v, cons
 }
 
 }  // namespace
+
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 unsigned long long wait_limit_ns() {
     // HYSPARSE_WAIT_LIMIT_NS lowers the bound on in-kernel waits; the tests
@@ -274,9 +280,18 @@ int hysparse_block(const hs_shape *shape, const void *q_full, const void *k, con
         rc = run_topk(s, scores, s.Lkv, r0, rows, topk, idx, st);
         if (rc != HS_OK) return rc;
     }
+    // the index set is shared by every sparse layer of the block, and so is
+    // the dense path's bitmask built from it
+    bool mask_ready = false;
+    if (n_sparse > 0 && prefer_dense_sparse(s, topk, window) && sparse_pair_supported(s)) {
+        uint32_t *mask = reinterpret_cast<uint32_t *>(w + ws_layout(s, topk, 1).selmask);
+        rc = cuda_status(selmask_build_launch(s, idx, topk, mask, reinterpret_cast<unsigned int *>(ws), st));
+        if (rc != HS_OK) return rc;
+        mask_ready = true;
+    }
     for (int n = 0; n < n_sparse; ++n) {
         rc = run_sparse(s, q_sparse[n], k, v, idx, topk, gate_logit[n], window, out_sparse[n],
-                        nullptr, nullptr, ws, st);
+                        nullptr, nullptr, ws, st, mask_ready);
         if (rc != HS_OK) return rc;
     }
     return HS_OK;
@@ -311,6 +326,8 @@ const char *hysparse_status_string(int status) {
 }
 
 const char *hysparse_version(void) { return "hysparse-b200 0.1"; }
+
+unsigned long long hysparse_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"
 

@@ -9,6 +9,10 @@
 
 namespace hs {
 
+// Number of kernels this library has launched (host-side count, exported for
+// benchmarks through hysparse_launch_count).
+void count_launch();
+
 // A validated hs_shape (scale resolved).
 struct Shape {
     int B, Lq, Lkv, Hq, Hkv, d;

@@ -244,7 +244,7 @@ cudaError_t launch_full_simt(const Shape &s, const void *q, const void *k, const
     dim3 grid(row_count, s.Hkv, s.B);
     kern<<<grid, 32 * G, sm, st>>>((const T *)q, (const T *)k, (const T *)v, (T *)out, lse, scores,
                                    ld, s.Lq, s.Lkv, s.Hq, s.Hkv, row_begin, row_count,
-                                   s.scale * kLog2e);
+                                   s.scale * kLog2e); count_launch();
     return cudaGetLastError();
 }
 
@@ -261,7 +261,7 @@ cudaError_t launch_sparse_simt(const Shape &s, const void *q, const void *k, con
     dim3 grid(s.Lq, s.Hkv, s.B);
     kern<<<grid, 32 * G, sm, st>>>((const T *)q, (const T *)k, (const T *)v, idx, topk, gate,
                                    window, (T *)out, (T *)og, (T *)ol, s.Lq, s.Lkv, s.Hq, s.Hkv,
-                                   s.scale * kLog2e, status);
+                                   s.scale * kLog2e, status); count_launch();
     return cudaGetLastError();
 }
 

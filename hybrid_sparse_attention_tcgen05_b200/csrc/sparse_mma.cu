@@ -491,10 +491,10 @@ cudaError_t launch_decode(const DecParams &dp, float *lse, float *scores, long l
     const long long items = (long long)dp.sp.B * dp.sp.Hkv * dp.nchunk;
     const long long blocks = (items + SW - 1) / SW;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-    decode_full_mma<NB><<<(unsigned)blocks, SW * 32, SpSmem<NB>::bytes, st>>>(dp);
+    decode_full_mma<NB><<<(unsigned)blocks, SW * 32, SpSmem<NB>::bytes, st>>>(dp); count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    decode_combine<<<dim3(dp.sp.Hkv, dp.sp.B), 256, 0, st>>>(dp, lse, scores, ld);
+    decode_combine<<<dim3(dp.sp.Hkv, dp.sp.B), 256, 0, st>>>(dp, lse, scores, ld); count_launch();
     return cudaGetLastError();
 }
 
@@ -510,7 +510,7 @@ cudaError_t launch_nb(const SpParams &p, cudaStream_t st) {
     const long long items = (long long)p.B * p.Lq * p.Hkv;
     const long long blocks = (items + SW - 1) / SW;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-    sparse_attn_mma<NB><<<(unsigned)blocks, SW * 32, SpSmem<NB>::bytes, st>>>(p);
+    sparse_attn_mma<NB><<<(unsigned)blocks, SW * 32, SpSmem<NB>::bytes, st>>>(p); count_launch();
     return cudaGetLastError();
 }
 

@@ -430,7 +430,7 @@ cudaError_t selmask_build_launch(const Shape &s, const int32_t *idx, int topk, u
     const long long mb = (n_rows + SM_WARPS - 1) / SM_WARPS;
     if (mb > 0x7fffffffLL) return cudaErrorInvalidValue;
     build_selmask<<<(unsigned)mb, SM_WARPS * 32, (size_t)SM_WARPS * W * 4, st>>>(idx, topk, s.Lq, s.Lkv, W, n_rows,
-                                                                                mask, status);
+                                                                                mask, status); count_launch();
     return cudaGetLastError();
 }
 
@@ -452,7 +452,7 @@ cudaError_t sparse_dense_tc_launch(const Shape &s, const void *q, const void *k,
     const long long mb = (n_rows + SM_WARPS - 1) / SM_WARPS;
     if (mb > 0x7fffffffLL) return cudaErrorInvalidValue;
     build_selmask<<<(unsigned)mb, SM_WARPS * 32, (size_t)SM_WARPS * W * 4, st>>>(idx, topk, s.Lq, s.Lkv, W, n_rows,
-                                                                                mask, status);
+                                                                                mask, status); count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     CUtensorMap mq, mk, mv;
@@ -462,7 +462,7 @@ cudaError_t sparse_dense_tc_launch(const Shape &s, const void *q, const void *k,
     SdParams p{s.Lq, s.Lkv, s.Hq, s.Hkv, s.G(), window, W, s.scale * kLog2e, mask, gate,
                (__nv_bfloat16 *)out, (__nv_bfloat16 *)og, (__nv_bfloat16 *)ol, status, wait_ns};
     const int n_tiles = (s.Lq + BM - 1) / BM;
-    sparse_dense_tc<<<dim3(n_tiles, s.Hq, s.B), SD_THREADS, kSdSmem, st>>>(mq, mk, mv, p);
+    sparse_dense_tc<<<dim3(n_tiles, s.Hq, s.B), SD_THREADS, kSdSmem, st>>>(mq, mk, mv, p); count_launch();
     return cudaGetLastError();
 }
 

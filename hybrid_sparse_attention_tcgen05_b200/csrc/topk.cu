@@ -190,13 +190,13 @@ cudaError_t topk_launch(const Shape &s, const float *scores, long long ld, int r
     if (split > 0) {
         const int n_max = off + row_begin + split;
         topk_radix_kernel<true><<<dim3(split, s.Hkv, s.B), NT, (size_t)n_max * 4, st>>>(
-            scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, 0, topk, idx);
+            scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, 0, topk, idx); count_launch();
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     if (split < row_count) {
         topk_radix_kernel<false><<<dim3(row_count - split, s.Hkv, s.B), NT, 0, st>>>(
-            scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, split, topk, idx);
+            scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, split, topk, idx); count_launch();
     }
     return cudaGetLastError();
 }

@@ -180,6 +180,10 @@ int hysparse_workspace_status(void *ws, hs_stream_t stream);
  * against exact 2^x.  Errors: HS_ERR_INVALID_ARG, HS_ERR_CUDA. */
 int hysparse_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int n, hs_stream_t stream);
 
+/* Diagnostic: number of CUDA kernels this library has launched in this
+ * process so far (counted on the host at each launch). */
+unsigned long long hysparse_launch_count(void);
+
 /* Static text for a status code. */
 const char *hysparse_status_string(int status);
 
