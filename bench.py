@@ -188,6 +188,22 @@ def work_model(w):
             "kv_bytes": kv_bytes, "keff": keff, "weff": weff, "pairs": P}
 
 
+def sparse_path_is_dense(w):
+    """The library's choice between the dense-masked and the gather sparse
+    kernel (same estimate as hysparse_api.cu; HYSPARSE_SPARSE_PATH overrides)."""
+    env = os.environ.get("HYSPARSE_SPARSE_PATH")
+    if w.dtype != "bf16" or w.Lq < 64:
+        return False
+    if env in ("dense", "gather"):
+        return env == "dense"
+    off = w.Lkv - w.Lq
+    tiles = sum(int((off + min(w.Lq, 128 * (t + 1)) - 1) // 128) + 1 for t in range((w.Lq + 127) // 128))
+    per_tile = 2600.0 if (w.Hq // w.Hkv) % 2 == 0 else 4000.0
+    dense_s = tiles * w.Hq * w.B * per_tile / (148.0 * 1.9e9)
+    gather_s = (sum_min(w, w.topk) + sum_min(w, w.window)) * w.Hkv * w.B * 512.0 / 6.0e12
+    return dense_s < gather_s
+
+
 # ------------------------------------------------------------------- ours
 
 def bench_ours(args, w, ws_, rank, local):
@@ -347,6 +363,7 @@ def bench_ours(args, w, ws_, rank, local):
 
     # ---- roofline of the dominant stage
     wm = work_model(w)
+    sparse_dense = sparse_path_is_dense(w)
     per = {kk: vv / args.steps for kk, vv in stage_ms.items()}
     dom = max(per, key=per.get)
     if dom == "full" and w.Lq == 1:
@@ -374,12 +391,25 @@ def bench_ours(args, w, ws_, rank, local):
         roof = {"kernel": "topk", "bound": "hbm", "unit": "GB/s",
                 "work": "4 B per causal (row, key, kv head) read + 4 B per index written"}
         key, srcs = "topk", ("topk.cu",)
+    elif sparse_dense:
+        # dense-masked tensor-core pass: report the method's useful FLOPs
+        # against the tensor peak; the executed (all causal tiles) rate beside it
+        launches = w.n_sparse
+        dur_s = per["sparse"] / launches / 1e3
+        useful = 4.0 * w.d * w.Hq * w.B * float(wm["keff"] + wm["weff"])
+        achieved = useful / dur_s / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"kernel": "sparse_attn (dense-masked: attn_fwd_tc<WIN>, attn_fwd_tc<SEL>, build_selmask)",
+                "bound": "tensor", "unit": "TFLOP/s",
+                "work": "4*d*Hq*(k_eff + w_eff) per row: the FLOPs the method needs",
+                "executed_tflops": wm["flops_full_fwd"] / dur_s / 1e12}
+        key, srcs = "sparse_pair", ("attn_tc.cu", "sparse_tc.cu")
     else:
         launches = w.n_sparse
         dur_s = per["sparse"] / launches / 1e3
         achieved = wm["gather_bytes_per_layer"] / dur_s / 1e9
         peak = peaks["hbm_gbs"]
-        roof = {"kernel": "sparse_attn", "bound": "hbm", "unit": "GB/s",
+        roof = {"kernel": "sparse_attn (gather: sparse_attn_mma)", "bound": "hbm", "unit": "GB/s",
                 "work": "(k_eff + w_eff) K and V rows per (row, kv head) + q, gate, out, idx"}
         key, srcs = "sparse_attn", ("sparse_mma.cu",)
     roof.update({"achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} (burst)",
