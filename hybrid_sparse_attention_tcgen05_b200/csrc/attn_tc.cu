@@ -19,12 +19,13 @@
 // group, so each K/V tile is loaded once for two Q tiles):
 //   warps 0-3  softmax for Q tile 0 (thread t owns row t = TMEM lane t)
 //   warps 4-7  softmax for Q tile 1
-//   warp 8     TMA producer (Q tiles once, then K_j, V_j through a 4-slot ring)
+//   warp 8     TMA producer (Q tiles once, then K and V tiles through a
+//              3-slot ring filled in the order the MMAs consume them)
 //   warp 9     MMA issuer (one thread)
-// TMEM (512 columns): S0 | S1 | O0 | O1, 128 f32 columns each.  P (bf16) is
-// written over the first 64 columns of its S tile and fed to the PV MMA
-// straight from TMEM.  MMAs issued by one thread execute in order, so
-// S_{j+1} = Q K_{j+1}^T may be issued right after O += P_j V_j.
+// TMEM (512 columns): S0 | S1 | O0 | O1, 128 f32 columns each.  P (bf16) goes
+// to shared memory in the swizzled layout of a Q tile, so the softmax
+// threads release S_j as soon as they have read it and S_{j+1} = Q K_{j+1}^T
+// runs on the tensor cores while they are still turning S_j into P_j.
 // The running max is only moved when it grows by more than 8 (log2 units);
 // the final normalisation uses the same reference, so the result is exact.
 #include <cuda.h>
