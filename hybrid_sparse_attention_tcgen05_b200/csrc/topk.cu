@@ -3,19 +3,26 @@
 // layer's TopK indices; baidu article "Top-K selection").
 //
 // Importance scores are sums of probabilities, so they are >= 0: the sign
-// bit is 0 and the other 31 bits, read as an unsigned integer, sort in the
-// same order as the values.  Three digit passes (bits 30-20, 19-10, 9-0) find
-// the exact bit pattern T of the k-th largest score and how many keys equal
-// to T must be taken; an ordered compaction then emits every key above T and
-// the lowest-indexed keys equal to T, which is exactly "largest scores, ties
-// to the lower index", already in ascending key order.  Integer work only:
-// the result is exact and deterministic.
+// bit is 0 and the 32-bit patterns, read as unsigned integers, sort in the
+// same order as the values.  With M the row's largest pattern and m its
+// smallest, every key has y = M - x in [0, M - m] < 2^L (L = bit length of
+// M - m), and the k largest scores are the k smallest y.  Digit passes over
+// y of at most 11 bits, most significant first (ceil(L / 11) passes: two for
+// the nearly flat rows of attention, whose keys share the exponent and the
+// leading mantissa bits), find the exact y_T of the k-th key and how many
+// keys equal to it must be taken; an ordered compaction then emits every key
+// above T = M - y_T and the lowest-indexed keys equal to T, which is exactly
+// "largest scores, ties to the lower index", already in ascending key order.
+// Integer work only: the result is exact and deterministic.
 //
-// Rows whose causal length fits (kSmemKeys) are first copied into shared
-// memory, so only that one read touches L2/HBM; longer rows are re-read from
-// global memory each pass.  The bin holding the k-th key is found by a
-// block-parallel scan over the bins (descending); the compaction uses
-// per-warp ballot counts and one pass over warp totals.
+// One CTA of 512 threads per (row, KV head).  The max / min pass copies the
+// row into shared memory when it is short enough to keep four CTAs on an SM;
+// longer rows are re-read from global memory (L2) by every pass, which
+// measured faster than a shared-memory copy at lower occupancy.  Keys are
+// read four at a time (16 bytes); histogram bins take plain shared atomics.
+#include <cstdlib>
+#include <cstring>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -24,56 +31,104 @@ namespace {
 
 constexpr int NT = 512;
 constexpr int NW = NT / 32;
-constexpr int kSmemKeys = 24576;       // 96 KB of row cache
-constexpr int kHistBins = 2048;
+constexpr unsigned int FULL = 0xffffffffu;
+constexpr int kDigitBits = 11;
+constexpr int kBins = 1 << kDigitBits;
+
+// Rows of up to kSmemKeys keys are cached in shared memory (39 KB + 16 KB of
+// histograms per CTA at the limit: four CTAs per SM).
+constexpr int kSmemKeys = 9984;
+
+// Launches with at least this many (row, KV head) items take the one-warp-
+// per-row kernel; fewer, longer rows (decode) take one CTA per row.
+constexpr long long kWarpMinItems = 4096;
 
 struct TopkShared {
-    unsigned int hist[kHistBins];
-    unsigned int sh_digit, sh_remaining;
-    unsigned int wsum[NW], woff[NW];
-    int cnt_gt[NW], cnt_eq[NW];
+    unsigned int h[2][kBins];      // digit histograms (passes alternate)
+    unsigned int wa[NW], wb[NW];   // per-warp partials
+    unsigned int digit, remaining;
 };
 
-// Find the bin (scanning from the top) in which the running count of keys
-// first reaches `remaining`; every thread owns nb / NT consecutive bins.
-// Writes the bin and the count still needed inside it to shared memory.
-__device__ __forceinline__ void find_bin(TopkShared &sh, unsigned int nb, unsigned int remaining, int tid) {
+// Keys 4g .. 4g+3 of the row (all four inside it).
+template <bool SMEM>
+__device__ __forceinline__ uint4 load4(const unsigned int *u, int g, bool aligned) {
+    if (SMEM) return reinterpret_cast<const uint4 *>(u)[g];
+    if (aligned) return __ldg(reinterpret_cast<const uint4 *>(u) + g);
+    const unsigned int *p = u + 4 * g;
+    return make_uint4(__ldg(p), __ldg(p + 1), __ldg(p + 2), __ldg(p + 3));
+}
+
+template <bool SMEM>
+__device__ __forceinline__ unsigned int load1(const unsigned int *u, int j) {
+    return SMEM ? u[j] : __ldg(u + j);
+}
+
+// One digit pass: key x takes part when the already fixed high bits of
+// y = M - x equal `pre` (y >> hs_ == pre; hs_ = 32: none fixed yet), and
+// falls into bin (y >> s) & nbm1.
+struct Digit {
+    unsigned int M, pre;
+    int hs_, s;
+    unsigned int nbm1;
+    __device__ __forceinline__ bool take(unsigned int x, unsigned int &bin) const {
+        const unsigned int y = M - x;
+        bin = (y >> s) & nbm1;
+        return hs_ >= 32 || (y >> hs_) == pre;
+    }
+};
+
+template <bool SMEM>
+__device__ __forceinline__ void hist_pass(unsigned int *hist, const unsigned int *u, int n, bool aligned,
+                                          const Digit &d, int tid) {
+    const int n4 = n >> 2;
+    for (int g = tid; g < n4; g += NT) {
+        const uint4 v = load4<SMEM>(u, g, aligned);
+        unsigned int b0, b1, b2, b3;
+        const bool t0 = d.take(v.x, b0), t1 = d.take(v.y, b1), t2 = d.take(v.z, b2), t3 = d.take(v.w, b3);
+        if (t0) atomicAdd(&hist[b0], 1u);
+        if (t1) atomicAdd(&hist[b1], 1u);
+        if (t2) atomicAdd(&hist[b2], 1u);
+        if (t3) atomicAdd(&hist[b3], 1u);
+    }
+    if (tid < n - 4 * n4) {
+        unsigned int bb;
+        if (d.take(load1<SMEM>(u, 4 * n4 + tid), bb)) atomicAdd(&hist[bb], 1u);
+    }
+}
+
+// Find the bin (ascending: smallest y first) in which the running count of
+// keys first reaches `remaining`; thread t owns bins per*t .. per*t+per-1.
+// Writes the bin and the count still needed inside it to sh.digit and
+// sh.remaining; the caller synchronises before reading them.
+__device__ __forceinline__ void find_bin(TopkShared &sh, const unsigned int *hist, unsigned int nb,
+                                         unsigned int remaining, int tid) {
     const int lane = tid & 31, warp = tid >> 5;
-    const int per = (int)nb / NT;
-    unsigned int c[kHistBins / NT];
+    const int per = nb >= (unsigned)NT ? (int)nb / NT : 1;
+    unsigned int c[kBins / NT];
     unsigned int tot = 0;
 #pragma unroll
-    for (int k = 0; k < kHistBins / NT; ++k) {
-        c[k] = k < per ? sh.hist[nb - 1 - (unsigned)(per * tid + k)] : 0u;
+    for (int k = 0; k < kBins / NT; ++k) {
+        const unsigned int bin = (unsigned)(per * tid + k);
+        c[k] = (k < per && bin < nb) ? hist[bin] : 0u;
         tot += c[k];
     }
     unsigned int incl = tot;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        const unsigned int y = __shfl_up_sync(0xffffffffu, incl, off);
+        const unsigned int y = __shfl_up_sync(FULL, incl, off);
         if (lane >= off) incl += y;
     }
-    if (lane == 31) sh.wsum[warp] = incl;
+    if (lane == 31) sh.wa[warp] = incl;
     __syncthreads();
-    if (warp == 0) {
-        unsigned int v = lane < NW ? sh.wsum[lane] : 0u;
-        unsigned int vi = v;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const unsigned int y = __shfl_up_sync(0xffffffffu, vi, off);
-            if (lane >= off) vi += y;
-        }
-        if (lane < NW) sh.woff[lane] = vi - v;
-    }
-    __syncthreads();
-    const unsigned int excl = sh.woff[warp] + incl - tot;
+    const unsigned int woff = __reduce_add_sync(FULL, lane < warp ? sh.wa[lane] : 0u);
+    const unsigned int excl = woff + incl - tot;
     if (excl < remaining && remaining <= excl + tot) {
         unsigned int cum = excl;
 #pragma unroll
-        for (int k = 0; k < kHistBins / NT; ++k) {
+        for (int k = 0; k < kBins / NT; ++k) {
             if (k < per && cum + c[k] >= remaining) {
-                sh.sh_digit = nb - 1 - (unsigned)(per * tid + k);
-                sh.sh_remaining = remaining - cum;
+                sh.digit = (unsigned)(per * tid + k);
+                sh.remaining = remaining - cum;
                 break;
             }
             cum += c[k];
@@ -82,11 +137,12 @@ __device__ __forceinline__ void find_bin(TopkShared &sh, unsigned int nb, unsign
 }
 
 template <bool SMEM>
-__global__ void __launch_bounds__(NT)
+__global__ void __launch_bounds__(NT, 4)
 topk_radix_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv, int Hkv, int row_begin,
                   int row_count, int r_lo, int topk, int32_t *__restrict__ idx) {
-    extern __shared__ unsigned int row_cache[];
+    extern __shared__ __align__(16) unsigned int row_cache[];
     __shared__ TopkShared sh;
+    __shared__ int cnt_gt[NW], cnt_eq[NW];
 
     const int r = r_lo + blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -100,72 +156,329 @@ topk_radix_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lk
         for (int t = tid; t < topk; t += NT) o[t] = t < n ? t : -1;
         return;
     }
-    const unsigned int *u = gu;
-    if (SMEM) {
-        for (int j = tid; j < n; j += NT) row_cache[j] = __ldg(gu + j);
-        __syncthreads();
-        u = row_cache;
-    }
+    const bool aligned = (reinterpret_cast<uintptr_t>(gu) & 15u) == 0;
+    for (int t = tid; t < 2 * kBins; t += NT) (&sh.h[0][0])[t] = 0u;
 
-    unsigned int prefix = 0, mask = 0, remaining = (unsigned int)topk;
-#pragma unroll
-    for (int ps = 0; ps < 3; ++ps) {
-        const int shift = ps == 0 ? 20 : (ps == 1 ? 10 : 0);
-        const unsigned int nb = ps == 0 ? 2048u : 1024u;
-        for (int t = tid; t < (int)nb; t += NT) sh.hist[t] = 0;
-        __syncthreads();
-        for (int j = tid; j < n; j += NT) {
-            const unsigned int x = SMEM ? u[j] : __ldg(u + j);
-            if ((x & mask) == prefix) atomicAdd(&sh.hist[(x >> shift) & (nb - 1u)], 1u);
+    // max / min bit pattern of the row (and its copy into shared memory)
+    unsigned int mx = 0u, mn = FULL;
+    const int n4 = n >> 2;
+    if (aligned) {
+        for (int q = tid; q < n4; q += NT) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(gu) + q);
+            if (SMEM) reinterpret_cast<uint4 *>(row_cache)[q] = v;
+            mx = max(mx, max(max(v.x, v.y), max(v.z, v.w)));
+            mn = min(mn, min(min(v.x, v.y), min(v.z, v.w)));
         }
-        __syncthreads();
-        find_bin(sh, nb, remaining, tid);
-        __syncthreads();
-        prefix |= sh.sh_digit << shift;
-        mask |= (nb - 1u) << shift;
-        remaining = sh.sh_remaining;
-        __syncthreads();
+    } else {
+        for (int j = tid; j < 4 * n4; j += NT) {
+            const unsigned int x = __ldg(gu + j);
+            if (SMEM) row_cache[j] = x;
+            mx = max(mx, x);
+            mn = min(mn, x);
+        }
     }
-
-    // prefix == the bit pattern of the k-th largest score.  Ordered
-    // compaction: warp w owns the contiguous key range [w*seg, (w+1)*seg).
-    // (A negative input, which importance scores never are, could only make
-    // more keys compare above T; the `at < topk` guard keeps writes in bounds.)
-    const unsigned int T = prefix;
-    const int seg = ((n + NW - 1) / NW + 31) & ~31;
-    const int j_lo = warp * seg, j_hi = min(n, j_lo + seg);
-    int gt = 0, eq = 0;
-    for (int j0 = j_lo; j0 < j_hi; j0 += 32) {
-        const int j = j0 + lane;
-        const unsigned int x = j < j_hi ? (SMEM ? u[j] : __ldg(u + j)) : 0u;
-        gt += __popc(__ballot_sync(0xffffffffu, j < j_hi && x > T));
-        eq += __popc(__ballot_sync(0xffffffffu, j < j_hi && x == T));
+    if (tid < n - 4 * n4) {
+        const unsigned int x = __ldg(gu + 4 * n4 + tid);
+        if (SMEM) row_cache[4 * n4 + tid] = x;
+        mx = max(mx, x);
+        mn = min(mn, x);
     }
+    mx = __reduce_max_sync(FULL, mx);
+    mn = __reduce_min_sync(FULL, mn);
     if (lane == 0) {
-        sh.cnt_gt[warp] = gt;
-        sh.cnt_eq[warp] = eq;
+        sh.wa[warp] = mx;
+        sh.wb[warp] = mn;
     }
     __syncthreads();
-    int gt_base = 0, eq_base = 0;
-    for (int w = 0; w < warp; ++w) {
-        gt_base += sh.cnt_gt[w];
-        eq_base += sh.cnt_eq[w];
+    const unsigned int M = __reduce_max_sync(FULL, lane < NW ? sh.wa[lane] : 0u);
+    const unsigned int range = M - __reduce_min_sync(FULL, lane < NW ? sh.wb[lane] : FULL);
+    const int L = range ? 32 - __clz(range) : 0;
+
+    const unsigned int *u = SMEM ? row_cache : gu;
+    const bool al = SMEM || aligned;
+
+    // digit passes over y = M - x, most significant first: after the pass
+    // covering bits [s, top), `pre` = y >> s of the k-th key
+    unsigned int pre = 0u, remaining = (unsigned int)topk;
+    int hs_ = 32, top = L, buf = 0;
+    while (top > 0) {
+        const int s = max(0, top - kDigitBits);
+        const unsigned int nb = 1u << (top - s);
+        const Digit d{M, pre, hs_, s, nb - 1u};
+        hist_pass<SMEM>(sh.h[buf], u, n, al, d, tid);
+        __syncthreads();
+        find_bin(sh, sh.h[buf], nb, remaining, tid);
+        __syncthreads();
+        pre = (pre << (top - s)) | sh.digit;
+        remaining = sh.remaining;
+        for (int t = tid; t < (int)nb; t += NT) sh.h[buf][t] = 0u;   // read by nobody until two passes on
+        hs_ = s;
+        top = s;
+        buf ^= 1;
     }
-    const unsigned int lt_mask = (1u << lane) - 1u;
-    for (int j0 = j_lo; j0 < j_hi; j0 += 32) {
-        const int j = j0 + lane;
-        const unsigned int x = j < j_hi ? (SMEM ? u[j] : __ldg(u + j)) : 0u;
-        const unsigned int bg = __ballot_sync(0xffffffffu, j < j_hi && x > T);
-        const unsigned int be = __ballot_sync(0xffffffffu, j < j_hi && x == T);
-        const int gtb = gt_base + __popc(bg & lt_mask);
-        const int eqb = eq_base + __popc(be & lt_mask);
-        const bool is_gt = (bg >> lane) & 1u, is_eq = (be >> lane) & 1u;
-        if (is_gt || (is_eq && eqb < (int)remaining)) {
-            const int at = gtb + min(eqb, (int)remaining);
-            if (at < topk) o[at] = j;
+    const unsigned int T = M - pre;   // bit pattern of the k-th largest score
+    const int rem = (int)remaining;   // keys equal to T to take (lowest indices first)
+
+    // Ordered compaction: warp w owns the contiguous key range
+    // [w*seg, (w+1)*seg), 128 keys (4 per lane) per step.  (A negative
+    // input, which importance scores never are, could only make more keys
+    // compare above T; the `at < topk` guard keeps writes in bounds.)
+    const int seg = ((n + NW - 1) / NW + 127) & ~127;
+    const int j_lo = warp * seg, j_hi = min(n, j_lo + seg);
+    int cg = 0, ce = 0;
+    for (int j = j_lo + 4 * lane; j < j_hi; j += 128) {
+        if (j + 4 <= j_hi) {
+            const uint4 v = load4<SMEM>(u, j >> 2, al);
+            cg += (v.x > T) + (v.y > T) + (v.z > T) + (v.w > T);
+            ce += (v.x == T) + (v.y == T) + (v.z == T) + (v.w == T);
+        } else {
+            for (int c = j; c < j_hi; ++c) {
+                const unsigned int x = load1<SMEM>(u, c);
+                cg += x > T;
+                ce += x == T;
+            }
         }
-        gt_base += __popc(bg);
-        eq_base += __popc(be);
+    }
+    cg = (int)__reduce_add_sync(FULL, (unsigned int)cg);
+    ce = (int)__reduce_add_sync(FULL, (unsigned int)ce);
+    if (lane == 0) {
+        cnt_gt[warp] = cg;
+        cnt_eq[warp] = ce;
+    }
+    __syncthreads();
+    int gt_base = (int)__reduce_add_sync(FULL, lane < warp ? (unsigned int)cnt_gt[lane] : 0u);
+    int eq_base = (int)__reduce_add_sync(FULL, lane < warp ? (unsigned int)cnt_eq[lane] : 0u);
+    for (int j0 = j_lo; j0 < j_hi; j0 += 128) {
+        const int j = j0 + 4 * lane;
+        const int nv = max(0, min(4, j_hi - j));
+        unsigned int xv[4] = {0u, 0u, 0u, 0u};
+        if (nv == 4) {
+            const uint4 v = load4<SMEM>(u, j >> 2, al);
+            xv[0] = v.x; xv[1] = v.y; xv[2] = v.z; xv[3] = v.w;
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (c < nv) xv[c] = load1<SMEM>(u, j + c);
+        }
+        bool isg[4], ise[4];
+        int ng = 0, ne = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            isg[c] = c < nv && xv[c] > T;
+            ise[c] = c < nv && xv[c] == T;
+            ng += isg[c];
+            ne += ise[c];
+        }
+        // exclusive lane prefix of (gt, eq) counts, packed 16:16 (<= 128 each)
+        const unsigned int packed = ((unsigned int)ng << 16) | (unsigned int)ne;
+        unsigned int incl = packed;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const unsigned int y = __shfl_up_sync(FULL, incl, off);
+            if (lane >= off) incl += y;
+        }
+        const unsigned int tot = __shfl_sync(FULL, incl, 31);
+        const unsigned int excl = incl - packed;
+        int gb = gt_base + (int)(excl >> 16), eb = eq_base + (int)(excl & 0xffffu);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (isg[c] || (ise[c] && eb < rem)) {
+                const int at = gb + min(eb, rem);
+                if (at < topk) o[at] = j + c;
+            }
+            gb += isg[c];
+            eb += ise[c];
+        }
+        gt_base += (int)(tot >> 16);
+        eq_base += (int)(tot & 0xffffu);
+    }
+}
+
+// ------------------------------------------------------------ one warp per row
+//
+// For launches with many rows (prefill): one warp owns one (row, KV head)
+// with a private 1024-bin histogram in shared memory, so the per-row fixed
+// work (histogram scans, clears) is one warp's and no block barrier is
+// needed; the compaction runs once over the row in key order (ballots give
+// each selected key its output slot), with no separate counting pass.  The
+// row is re-read from global memory (L1 / L2) by each of its passes.
+
+constexpr int WK_WARPS = 8;
+constexpr int WK_BITS = 10;
+constexpr int WK_BINS = 1 << WK_BITS;
+
+template <bool AL>
+__device__ __forceinline__ uint4 ld4(const unsigned int *u, int g) {
+    if (AL) return __ldg(reinterpret_cast<const uint4 *>(u) + g);
+    const unsigned int *p = u + 4 * g;
+    return make_uint4(__ldg(p), __ldg(p + 1), __ldg(p + 2), __ldg(p + 3));
+}
+
+__device__ __forceinline__ void wk_zero(unsigned int *h, int lane) {
+#pragma unroll
+    for (int k = 0; k < WK_BINS / 128; ++k)
+        reinterpret_cast<uint4 *>(h)[k * 32 + lane] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// Smallest bin b (ascending) whose running count reaches `remaining`;
+// returns b, the count still needed inside it and the bin's own count.
+__device__ __forceinline__ unsigned int wk_find(const unsigned int *h, unsigned int remaining, int lane,
+                                                unsigned int &rem_out, unsigned int &cnt_out) {
+    // lane l sums bins [32l, 32l+32), reading them in a rotated order so the
+    // 32 lanes hit 32 different banks
+    unsigned int tot = 0;
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) tot += h[32 * lane + ((k + lane) & 31)];
+    unsigned int incl = tot;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const unsigned int y = __shfl_up_sync(FULL, incl, off);
+        if (lane >= off) incl += y;
+    }
+    const int c = max(0, __ffs(__ballot_sync(FULL, incl >= remaining)) - 1);   // chunk holding the k-th key
+    const unsigned int before = __shfl_sync(FULL, incl - tot, c);
+    const unsigned int v = h[32 * c + lane];
+    unsigned int in2 = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const unsigned int y = __shfl_up_sync(FULL, in2, off);
+        if (lane >= off) in2 += y;
+    }
+    const int e = max(0, __ffs(__ballot_sync(FULL, before + in2 >= remaining)) - 1);
+    rem_out = remaining - before - __shfl_sync(FULL, in2 - v, e);
+    cnt_out = __shfl_sync(FULL, v, e);
+    return (unsigned int)(32 * c + e);
+}
+
+template <bool AL>
+__global__ void __launch_bounds__(WK_WARPS * 32, 5)
+topk_warp_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv, int Hkv, int row_begin,
+                 int row_count, int topk, long long n_items, int32_t *__restrict__ idx) {
+    __shared__ __align__(16) unsigned int hist_all[WK_WARPS][WK_BINS];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long item = (long long)blockIdx.x * WK_WARPS + warp;
+    if (item >= n_items) return;
+    // longest rows first; (batch, KV head) slowest
+    const int r = row_count - 1 - (int)(item % row_count);
+    const long long bg = item / row_count;
+    const int i = row_begin + r;
+    const int n = Lkv - Lq + i + 1;
+    const unsigned int *u = reinterpret_cast<const unsigned int *>(scores + ((size_t)bg * row_count + r) * ld);
+    int32_t *o = idx + ((size_t)bg * Lq + i) * (size_t)topk;
+    if (n <= topk) {
+        for (int t = lane; t < topk; t += 32) o[t] = t < n ? t : -1;
+        return;
+    }
+    unsigned int *h = hist_all[warp];
+    wk_zero(h, lane);
+
+    const int n4 = n >> 2, nt = n - 4 * n4;
+    const unsigned int xt = lane < nt ? __ldg(u + 4 * n4 + lane) : 0u;   // tail keys (< 4)
+    unsigned int mx = lane < nt ? xt : 0u, mn = lane < nt ? xt : FULL;
+    for (int g = lane; g < n4; g += 32) {
+        const uint4 v = ld4<AL>(u, g);
+        mx = max(mx, max(max(v.x, v.y), max(v.z, v.w)));
+        mn = min(mn, min(min(v.x, v.y), min(v.z, v.w)));
+    }
+    const unsigned int M = __reduce_max_sync(FULL, mx);
+    const unsigned int range = M - __reduce_min_sync(FULL, mn);
+    const int L = range ? 32 - __clz(range) : 0;
+    __syncwarp();
+
+    unsigned int pre = 0u, remaining = (unsigned int)topk, cnt_eq = (unsigned int)n;
+    int hs_ = 32, top = L;
+    while (top > 0) {
+        const int s = max(0, top - WK_BITS);
+        const unsigned int msk = (1u << (top - s)) - 1u;
+        if (hs_ >= 32) {
+            for (int g = lane; g < n4; g += 32) {
+                const uint4 v = ld4<AL>(u, g);
+                atomicAdd(&h[(M - v.x) >> s], 1u);
+                atomicAdd(&h[(M - v.y) >> s], 1u);
+                atomicAdd(&h[(M - v.z) >> s], 1u);
+                atomicAdd(&h[(M - v.w) >> s], 1u);
+            }
+            if (lane < nt) atomicAdd(&h[(M - xt) >> s], 1u);
+        } else {
+            for (int g = lane; g < n4; g += 32) {
+                const uint4 v = ld4<AL>(u, g);
+                const unsigned int y0 = M - v.x, y1 = M - v.y, y2 = M - v.z, y3 = M - v.w;
+                if ((y0 >> hs_) == pre) atomicAdd(&h[(y0 >> s) & msk], 1u);
+                if ((y1 >> hs_) == pre) atomicAdd(&h[(y1 >> s) & msk], 1u);
+                if ((y2 >> hs_) == pre) atomicAdd(&h[(y2 >> s) & msk], 1u);
+                if ((y3 >> hs_) == pre) atomicAdd(&h[(y3 >> s) & msk], 1u);
+            }
+            if (lane < nt && ((M - xt) >> hs_) == pre) atomicAdd(&h[((M - xt) >> s) & msk], 1u);
+        }
+        __syncwarp();
+        unsigned int rem2, cnt;
+        const unsigned int dig = wk_find(h, remaining, lane, rem2, cnt);
+        __syncwarp();
+        wk_zero(h, lane);
+        __syncwarp();
+        pre = (pre << (top - s)) | dig;
+        remaining = rem2;
+        cnt_eq = cnt;
+        hs_ = s;
+        top = s;
+    }
+    const unsigned int T = M - pre;            // bit pattern of the k-th largest score
+    const bool take_all = remaining == cnt_eq; // every key equal to T is taken: no tie ranks needed
+    const unsigned int lt = (1u << lane) - 1u;
+    int base = 0, eq_base = 0;
+    for (int g0 = 0; g0 < n4 + 1; g0 += 32) {   // the extra step carries the tail keys
+        const int g = g0 + lane;
+        unsigned int x[4];
+        bool ok[4];
+        if (g < n4) {
+            const uint4 v = ld4<AL>(u, g);
+            x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+            ok[0] = ok[1] = ok[2] = ok[3] = true;
+        } else {
+            const int tail0 = 4 * n4 + 4 * (g - n4);   // tail keys sit in group n4 only
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                ok[c] = g == n4 && c < nt;
+                x[c] = ok[c] ? __ldg(u + tail0 + c) : 0u;
+            }
+        }
+        bool sel[4];
+        if (take_all) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) sel[c] = ok[c] && x[c] >= T;
+        } else {
+            bool eq[4];
+            int eq_lane = 0;
+            unsigned int eb_all = 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                eq[c] = ok[c] && x[c] == T;
+                const unsigned int bb = __ballot_sync(FULL, eq[c]);
+                eq_lane += __popc(bb & lt);
+                eb_all += __popc(bb);
+            }
+            int er = eq_base + eq_lane;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                sel[c] = (ok[c] && x[c] > T) || (eq[c] && er < (int)remaining);
+                er += eq[c];
+            }
+            eq_base += (int)eb_all;
+        }
+        int before = 0, tot = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const unsigned int bb = __ballot_sync(FULL, sel[c]);
+            before += __popc(bb & lt);
+            tot += __popc(bb);
+        }
+        int at = base + before;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (sel[c] && at < topk) o[at] = 4 * g + c;
+            at += sel[c];
+        }
+        base += tot;
     }
 }
 
@@ -180,23 +493,40 @@ cudaError_t topk_launch(const Shape &s, const float *scores, long long ld, int r
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    // rows are ordered by causal length; those up to kSmemKeys keys run with
-    // the row cached in shared memory, sized for the longest of them
-    const int off = s.Lkv - s.Lq;
-    const int n_first = off + row_begin + 1;
-    int split = row_count;                                   // rows [0, split) fit
-    if (n_first > kSmemKeys) split = 0;
-    else if (off + row_begin + row_count > kSmemKeys) split = kSmemKeys - off - row_begin;
+    const long long n_items = (long long)s.B * s.Hkv * row_count;
+    // HYSPARSE_TOPK_PATH=warp|block forces one kernel (the tests run both)
+    const char *force = getenv("HYSPARSE_TOPK_PATH");
+    const bool use_warp = force && strcmp(force, "warp") == 0    ? true
+                          : force && strcmp(force, "block") == 0 ? false
+                                                                 : n_items >= kWarpMinItems;
+    if (use_warp) {
+        const bool al = (reinterpret_cast<uintptr_t>(scores) & 15u) == 0 && (ld & 3) == 0;
+        const unsigned int grid = (unsigned int)((n_items + WK_WARPS - 1) / WK_WARPS);
+        if (al)
+            topk_warp_kernel<true><<<grid, WK_WARPS * 32, 0, st>>>(scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin,
+                                                                   row_count, topk, n_items, idx);
+        else
+            topk_warp_kernel<false><<<grid, WK_WARPS * 32, 0, st>>>(scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin,
+                                                                    row_count, topk, n_items, idx);
+        count_launch();
+        return cudaGetLastError();
+    }
+    // Few rows (decode): one CTA per row.  Rows are ordered by causal length
+    // n = off + row_begin + r + 1: those with n <= kSmemKeys run with the row
+    // cached in shared memory (sized for the longest of them), the rest read
+    // global memory.
+    const long long off = (long long)s.Lkv - s.Lq;
+    const long long split = max(0ll, min((long long)row_count, (long long)kSmemKeys - off - row_begin));
     if (split > 0) {
-        const int n_max = off + row_begin + split;
-        topk_radix_kernel<true><<<dim3(split, s.Hkv, s.B), NT, (size_t)n_max * 4, st>>>(
+        const long long n_max = off + row_begin + split;
+        topk_radix_kernel<true><<<dim3((unsigned)split, s.Hkv, s.B), NT, (size_t)n_max * 4, st>>>(
             scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, 0, topk, idx); count_launch();
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     if (split < row_count) {
-        topk_radix_kernel<false><<<dim3(row_count - split, s.Hkv, s.B), NT, 0, st>>>(
-            scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, split, topk, idx); count_launch();
+        topk_radix_kernel<false><<<dim3((unsigned)(row_count - split), s.Hkv, s.B), NT, 0, st>>>(
+            scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, (int)split, topk, idx); count_launch();
     }
     return cudaGetLastError();
 }

@@ -124,30 +124,50 @@ def test_topk_stage_isolated_bit_exact():
     assert torch.equal(idx[0, 0].cpu(), o_idx)
 
 
-@pytest.mark.parametrize("case", ["ties", "all_equal", "zeros_and_denormals", "long_rows", "split_rows",
-                                  "flat_narrow"])
-def test_topk_synthetic_rows_bit_exact(case):
-    """Score rows built directly (not by the CUDA path), with exact ties."""
+# Row lengths around which the top-k launch switches from rows cached in
+# shared memory to rows read from global memory (and a few other lengths).
+TOPK_BUCKET_EDGES = (9984, 25600)
+
+
+@pytest.mark.parametrize("case", ["ties", "ties_unaligned", "all_equal", "zeros_and_denormals", "long_rows",
+                                  "flat_narrow", "flat_long_unaligned", "many_rows_ties"]
+                         + [f"edge{e}" for e in TOPK_BUCKET_EDGES]
+                         + [f"edge{e}_unaligned" for e in TOPK_BUCKET_EDGES])
+@pytest.mark.parametrize("kernel", ["block", "warp"])
+def test_topk_synthetic_rows_bit_exact(case, kernel, monkeypatch):
+    """Score rows built directly (not by the CUDA path), with exact ties,
+    through both top-k kernels (one CTA per row / one warp per row)."""
+    monkeypatch.setenv("HYSPARSE_TOPK_PATH", kernel)
     g = torch.Generator().manual_seed(7)
     B, Hkv, Lq, Lkv, k = 2, 3, 37, 300, 29
     if case == "long_rows":
         Lq, Lkv, k = 5, 70000, 2048
-    elif case == "split_rows":      # rows on both sides of the shared-memory row-cache limit
-        Lq, Lkv, k = 40, 24600, 1000
+    elif case.startswith("edge"):    # rows on both sides of a bucket edge
+        e = int(case[4:].split("_")[0])
+        B, Hkv, Lq, k = 1, 2, 40, 1000
+        Lkv = e + 20 + (1 if case.endswith("unaligned") else 0)   # odd Lkv: rows not 16-byte aligned
     elif case == "flat_narrow":     # near-flat rows: every key in one coarse bin
         Lq, Lkv, k = 16, 20000, 1500
+    elif case == "flat_long_unaligned":
+        B, Hkv, Lq, Lkv, k = 1, 1, 6, 60001, 2048
+    elif case == "ties_unaligned":
+        Lkv = 301
+    elif case == "many_rows_ties":   # enough rows for the one-warp-per-row kernel by default
+        B, Hkv, Lq, Lkv, k = 1, 2, 2100, 2203, 150
     s = torch.rand(B, Hkv, Lq, Lkv, generator=g)
-    if case == "ties":
+    if case in ("ties", "ties_unaligned"):
         s = torch.round(s * 16) / 16
+    elif case == "many_rows_ties":
+        s = torch.round(s * 512) / 512
     elif case == "all_equal":
         s[:] = 0.125
     elif case == "zeros_and_denormals":
         s = torch.where(s < 0.5, torch.zeros_like(s), s * 1e-39)
     elif case == "long_rows":
         s = torch.round(s * 4096) / 4096
-    elif case == "split_rows":
+    elif case.startswith("edge"):
         s = torch.round(s * 65536) / 65536
-    elif case == "flat_narrow":
+    elif case.startswith("flat"):
         s = (1.0 + 0.02 * s) / 8192.0
     shape = hs.HsShape(B, Lq, Lkv, 4 * Hkv, Hkv, 128, 1, 0.0)
     idx = hs.topk(shape, s.to(DEV), k)
