@@ -28,6 +28,8 @@
 // runs on the tensor cores while they are still turning S_j into P_j.
 // The running max is only moved when it grows by more than 8 (log2 units);
 // the final normalisation uses the same reference, so the result is exact.
+#include <cstring>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -44,10 +46,11 @@ namespace {
 // Share of the softmax exponentials computed by exp2_poly on the FMA pipe
 // instead of the MUFU unit: every kFwdPolyEvery-th element of the forward
 // pass, every kScPolyEvery-th of the score pass (0 = none).  Measured on
-// B200: the score pass is MUFU-bound and gains ~1.5 % at 1/4 (more hurts);
-// the forward pass is not MUFU-bound and only loses, so it stays at 0.
+// B200 with the packed f32x2 FMAs: both passes are fastest with every
+// exponential on the MUFU unit (the polynomial's instructions cost more
+// issue slots than the MUFU time they free).
 constexpr int kFwdPolyEvery = 0;
-constexpr int kScPolyEvery = 4;
+constexpr int kScPolyEvery = 0;
 
 constexpr int FWD_KV = 3;   // K/V ring slots (shared memory also holds Q0, Q1, P0, P1)
 
@@ -297,8 +300,13 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                     if (j0 + c > pos) s[c] = -INFINITY;
             }
             float m4[4] = {s[0], s[1], s[2], s[3]};
+            if (MODE == FWD_FULL) {
 #pragma unroll
-            for (int c = 4; c < 128; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
+                for (int c = 4; c < 128; c += 2) m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], s[c], s[c + 1]);
+            } else {   // measured: the two-input chain is faster in the masked modes
+#pragma unroll
+                for (int c = 4; c < 128; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
+            }
             const float mx2 = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c2;
             // PV of the previous tile done: O is stable and the P buffer is free
             if (j > 0) {
@@ -327,17 +335,25 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                 m = m_new;
             }
             const float mref = m == -INFINITY ? 0.f : m;   // masked keys (-inf) give 2^-inf = 0
-            float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
+            const float2 c2v = make_float2(c2, c2), mv = make_float2(-mref, -mref);
+            float2 ps01 = make_float2(0.f, 0.f), ps23 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int ch = 0; ch < 16; ++ch) {           // 16-byte chunks of 8 keys
                 uint32_t pk[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int c = ch * 8 + 2 * e;
-                    const float a = ex2_mix<kFwdPolyEvery>(fmaf(s[c], c2, -mref), c);
-                    const float bb = ex2_mix<kFwdPolyEvery>(fmaf(s[c + 1], c2, -mref), c + 1);
-                    if (e & 1) { ps2 += a; ps3 += bb; } else { ps0 += a; ps1 += bb; }
-                    pk[e] = pack_bf16(a, bb);
+                    float2 ab;
+                    if (MODE != FWD_FULL) {   // measured: packed pairs spill or lose in the masked modes
+                        ab = make_float2(ex2_mix<kFwdPolyEvery>(fmaf(s[c], c2, -mref), c),
+                                         ex2_mix<kFwdPolyEvery>(fmaf(s[c + 1], c2, -mref), c + 1));
+                        if (e & 1) { ps23.x += ab.x; ps23.y += ab.y; } else { ps01.x += ab.x; ps01.y += ab.y; }
+                    } else {
+                        const float2 t = ffma2(make_float2(s[c], s[c + 1]), c2v, mv);
+                        ab = make_float2(ex2_mix<kFwdPolyEvery>(t.x, c), ex2_mix<kFwdPolyEvery>(t.y, c + 1));
+                        if (e & 1) ps23 = fadd2(ps23, ab); else ps01 = fadd2(ps01, ab);
+                    }
+                    pk[e] = pack_bf16(ab.x, ab.y);
                 }
                 const int half = ch >> 3, c8 = ch & 7;
                 *reinterpret_cast<uint4 *>(prow + half * HALF + ((c8 ^ sw) << 4)) =
@@ -345,7 +361,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             }
             fence_proxy_async_smem();
             mbar_arrive(smem_u32(&bars->p_full[w]));
-            const float ts = (ps0 + ps1) + (ps2 + ps3);
+            const float ts = (ps01.x + ps01.y) + (ps23.x + ps23.y);
             const float y = ts - lc;
             const float t = l + y;
             lc = (t - l) - y;
@@ -456,10 +472,17 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 
 // ------------------------------------------------------------------ scores
 
-constexpr int SC_Q_STAGES = 5;   // Q slots: all G query tiles stay resident when G <= 5, else a ring
+constexpr int SC_Q_STAGES = 4;   // Q slots: all G query tiles stay resident when G <= 4, else a ring
 constexpr int SC_K_STAGES = 2;
 constexpr int SC_BUFS = 4;
-constexpr int SC_THREADS = 320;   // warps 0-7 scores (two per lane quarter), 8 TMA, 9 MMA
+// warps 0-15 scores (four per TMEM lane quarter, 32 columns each), 16 TMA, 17 MMA
+constexpr int SC_SCORE_WARPS = 16;
+constexpr int SC_TMA_WARP = SC_SCORE_WARPS, SC_MMA_WARP = SC_SCORE_WARPS + 1;
+constexpr int SC_THREADS = 32 * (SC_SCORE_WARPS + 2);
+// Score staging for the bulk tensor stores: per score warp one 2 KB buffer,
+// a 32-row x 16-column fp32 box in the 64-byte swizzled layout.
+constexpr int SC_STG_BYTES = 2048;
+constexpr int SC_STG_TOTAL = SC_SCORE_WARPS * SC_STG_BYTES;
 
 struct ScBars {
     uint64_t q_full[SC_Q_STAGES], q_empty[SC_Q_STAGES];
@@ -470,7 +493,7 @@ struct ScBars {
     int abort;
 };
 
-constexpr size_t kScSmem = 1024 + (SC_Q_STAGES + SC_K_STAGES) * TILE + sizeof(ScBars);
+constexpr size_t kScSmem = 1024 + (SC_Q_STAGES + SC_K_STAGES) * TILE + SC_STG_TOTAL + sizeof(ScBars);
 
 struct ScParams {
     int Lq, Lkv, Hq, Hkv, G;
@@ -481,16 +504,18 @@ struct ScParams {
     long long ld;
     unsigned int *status;
     unsigned long long wait_ns;
+    int tma_store;   // scores leave through `ts` (bulk tensor stores) rather than per-thread stores
 };
 
 __global__ void __launch_bounds__(SC_THREADS, 1)
 attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-               const ScParams p) {
+               const __grid_constant__ CUtensorMap ts, const ScParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     uint8_t *sq = smem;
     uint8_t *sk = smem + SC_Q_STAGES * TILE;
-    ScBars *bars = reinterpret_cast<ScBars *>(smem + (SC_Q_STAGES + SC_K_STAGES) * TILE);
+    uint8_t *sst = smem + (SC_Q_STAGES + SC_K_STAGES) * TILE;
+    ScBars *bars = reinterpret_cast<ScBars *>(sst + SC_STG_TOTAL);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tile = gridDim.x - 1 - blockIdx.x;
@@ -515,7 +540,7 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         }
         for (int s = 0; s < SC_BUFS; ++s) {
             mbar_init(smem_u32(&bars->s_full[s]), 1);
-            mbar_init(smem_u32(&bars->s_free[s]), 256);
+            mbar_init(smem_u32(&bars->s_free[s]), 32 * SC_SCORE_WARPS);
         }
         mbar_init(smem_u32(&bars->drain), 1);
         bars->abort = 0;
@@ -531,7 +556,7 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     const uint32_t tmem = bars->tmem_base;
     volatile int *abort = &bars->abort;
 
-    if (warp == 8) {
+    if (warp == SC_TMA_WARP) {
         if (lane == 0) {
             tma_prefetch(&tq);
             tma_prefetch(&tk);
@@ -572,7 +597,7 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     mbar_drain(smem_u32(&bars->q_full[it % SC_Q_STAGES]), (it / SC_Q_STAGES) & 1);
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == SC_MMA_WARP) {
         if (lane == 0) {
             bool ok = true;
             for (int j = 0; ok && j < n_kv; ++j) {
@@ -599,64 +624,97 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         }
     } else {
         // ------------------------------------------------ score warps
-        // warp w serves TMEM lanes 32*(w%4).. and columns 64*(w/4) .. +63
-        const int q4 = warp & 3, half = warp >> 2;
+        // warp w serves TMEM lanes 32*(w%4) .. +31 and columns 32*(w/4) .. +31
+        const int q4 = warp & 3, cq = warp >> 2;
         const int tw = 32 * q4 + lane;
         const int row = r0 + tw;
         const bool valid = row < r_end;
         const int pos = off + min(row, r_end - 1);
         const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-        const uint32_t colh = (uint32_t)(64 * half);
+        const uint32_t colq = (uint32_t)(32 * cq);
         const float c2 = p.scale_log2;
         float *srow = valid ? p.scores + (((size_t)b * p.Hkv + g) * p.row_count + (row - p.row_begin)) * p.ld
                             : nullptr;
         const bool vec4 = (p.ld & 3) == 0;
+        uint8_t *stg = sst + warp * SC_STG_BYTES;
+        const int srow0 = r0 - p.row_begin + 32 * q4;       // this warp's first row within the chunk
+        const int zbg = b * p.Hkv + g;
+        const int sw = (lane >> 1) & 3;                      // 64-byte swizzle phase of this thread's row
+        // the per-(row, head) statistics are loaded one head ahead
+        const size_t st0 = ((size_t)b * p.Hq + (size_t)g * G) * p.Lq + row;
+        float2 st_next = valid ? p.stats[st0] : make_float2(0.f, 0.f);
         bool ok = true;
         for (int j = 0; ok && j < n_kv; ++j) {
-            float acc[64];
+            float acc[32];
 #pragma unroll
-            for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+            for (int c = 0; c < 32; ++c) acc[c] = 0.f;
             for (int hh = 0; hh < G; ++hh) {
                 const int it = j * G + hh, buf = it % SC_BUFS;
-                const float2 st = valid ? p.stats[((size_t)b * p.Hq + g * G + hh) * p.Lq + row]
-                                        : make_float2(0.f, 0.f);
+                const float2 st = st_next;
+                const int hn = hh + 1 < G ? hh + 1 : 0;
+                if (valid) st_next = p.stats[st0 + (size_t)hn * p.Lq];
                 ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[buf]), (it / SC_BUFS) & 1, p.wait_ns, abort));
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t tS = tmem + lane_off + (uint32_t)(buf * 128) + colh;
-                uint32_t r[2][32];
-                tmem_ld32(tS, r[0]);
-                tmem_ld32(tS + 32, r[1]);
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_off + (uint32_t)(buf * 128) + colq, r);
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(smem_u32(&bars->s_free[buf]));   // S is in registers; the MMA may reuse the buffer
+                const float2 c2v = make_float2(c2, c2), mv = make_float2(-st.x, -st.x), lv = make_float2(st.y, st.y);
 #pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    acc[c] = fmaf(ex2_mix<kScPolyEvery>(fmaf(__uint_as_float(r[c >> 5][c & 31]), c2, -st.x), c),
-                                  st.y, acc[c]);
+                for (int c = 0; c < 32; c += 2) {
+                    const float2 t = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), c2v, mv);
+                    const float2 e = make_float2(ex2_mix<kScPolyEvery>(t.x, c), ex2_mix<kScPolyEvery>(t.y, c + 1));
+                    const float2 a2 = ffma2(e, lv, make_float2(acc[c], acc[c + 1]));
+                    acc[c] = a2.x;
+                    acc[c + 1] = a2.y;
+                }
             }
             if (!ok) break;
-            if (valid) {
-                const int j0 = j * BN + 64 * half;
-                const int lim = min(64, p.Lkv - j0);      // columns inside the cache
-                const int keep = min(lim, pos - j0 + 1);  // causal columns
+            const int j0 = j * BN + 32 * cq;
+            const int keep = pos - j0 + 1;                  // causal columns of this row in the 32
+            if (p.tma_store) {
+                // 2 boxes of 32 rows x 16 columns through the staging buffer
+#pragma unroll
+                for (int rnd = 0; rnd < 2; ++rnd) {
+                    if (lane == 0) bulk_wait_read<0>();     // the previous store has read the buffer
+                    __syncwarp();
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const int c = 16 * rnd + 4 * c4;
+                        const float4 v4 = make_float4(c < keep ? acc[c] : 0.f, c + 1 < keep ? acc[c + 1] : 0.f,
+                                                      c + 2 < keep ? acc[c + 2] : 0.f, c + 3 < keep ? acc[c + 3] : 0.f);
+                        *reinterpret_cast<float4 *>(stg + lane * 64 + ((c4 ^ sw) << 4)) = v4;
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    const int x0 = j0 + 16 * rnd;
+                    if (lane == 0 && x0 < p.Lkv && srow0 < p.row_count) {
+                        tma_store_3d(&ts, smem_u32(stg), x0, srow0, zbg);
+                        bulk_commit();
+                    }
+                }
+            } else if (valid) {
+                const int lim = min(32, p.Lkv - j0);      // columns inside the cache
                 float *dst = srow + j0;
                 if (lim > 0) {
-                    if (vec4 && lim == 64) {
+                    if (vec4 && lim == 32) {
 #pragma unroll
-                        for (int c = 0; c < 64; c += 4) {
+                        for (int c = 0; c < 32; c += 4) {
                             float4 v4 = make_float4(c < keep ? acc[c] : 0.f, c + 1 < keep ? acc[c + 1] : 0.f,
                                                     c + 2 < keep ? acc[c + 2] : 0.f, c + 3 < keep ? acc[c + 3] : 0.f);
                             *reinterpret_cast<float4 *>(dst + c) = v4;
                         }
                     } else {
 #pragma unroll
-                        for (int c = 0; c < 64; ++c)
+                        for (int c = 0; c < 32; ++c)
                             if (c < lim) dst[c] = c < keep ? acc[c] : 0.f;
                     }
                 }
             }
         }
+        if (p.tma_store && lane == 0) bulk_wait_all();   // scores written before the CTA retires
     }
 
     tc_fence_before();
@@ -705,8 +763,23 @@ cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || scores == nullptr) return e;
     ScParams sp{s.Lq, s.Lkv, s.Hq, s.Hkv, s.G(), row_begin, row_begin + row_count, row_count,
-                s.scale * kLog2e, stats, scores, ld, status, wait_ns};
-    attn_scores_tc<<<dim3(n_tiles, s.Hkv, s.B), SC_THREADS, kScSmem, st>>>(mq, mk, sp); count_launch();
+                s.scale * kLog2e, stats, scores, ld, status, wait_ns, 0};
+    // scores [B][Hkv][row_count][ld] f32 as a 3-D map (key, row, batch*KV head)
+    // with 16 x 32 boxes in the 64-byte swizzle; needs 16-byte aligned rows
+    CUtensorMap ms;
+    memset(&ms, 0, sizeof(ms));
+    if ((ld & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15u) == 0) {
+        auto enc = encode_fn();
+        cuuint64_t dims[3] = {(cuuint64_t)s.Lkv, (cuuint64_t)row_count, (cuuint64_t)s.B * s.Hkv};
+        cuuint64_t strides[2] = {(cuuint64_t)ld * 4, (cuuint64_t)ld * 4 * row_count};
+        cuuint32_t box[3] = {16, 32, 1};
+        cuuint32_t es[3] = {1, 1, 1};
+        if (enc && enc(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, scores, dims, strides, box, es,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+            sp.tma_store = 1;
+    }
+    attn_scores_tc<<<dim3(n_tiles, s.Hkv, s.B), SC_THREADS, kScSmem, st>>>(mq, mk, ms, sp); count_launch();
     return cudaGetLastError();
 }
 
