@@ -123,12 +123,12 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     FwdBars *bars = reinterpret_cast<FwdBars *>(smem + 4 * TILE + FWD_KV * TILE);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tile = gridDim.x - 1 - blockIdx.x;  // heaviest row tiles first
+    int tile, b;
+    tile_of_block((p.row_end - p.row_begin + BM - 1) / BM, tile, b);   // heaviest row tiles first
     const int r0 = p.row_begin + tile * BM;
     const int r_end = min(r0 + BM, p.row_end);
-    const int h0 = 2 * blockIdx.y;
+    const int h0 = 2 * blockIdx.x;
     const int g = h0 / p.G;
-    const int b = blockIdx.z;
     const int off = p.Lkv - p.Lq;
     const int pos_first = off + r0;
     const int pos_last = off + r_end - 1;
@@ -518,11 +518,11 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     ScBars *bars = reinterpret_cast<ScBars *>(sst + SC_STG_TOTAL);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tile = gridDim.x - 1 - blockIdx.x;
+    int tile, b;
+    tile_of_block((p.row_end - p.row_begin + BM - 1) / BM, tile, b);   // heaviest row tiles first
     const int r0 = p.row_begin + tile * BM;
     const int r_end = min(r0 + BM, p.row_end);
-    const int g = blockIdx.y;
-    const int b = blockIdx.z;
+    const int g = blockIdx.x;
     const int G = p.G;
     const bool resident = G <= SC_Q_STAGES;
     const int off = p.Lkv - p.Lq;
@@ -759,7 +759,7 @@ cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void
     fp.row_begin = row_begin; fp.row_end = row_begin + row_count;
     fp.scale_log2 = s.scale * kLog2e;
     fp.out = (__nv_bfloat16 *)out; fp.lse = lse; fp.stats = stats; fp.status = status; fp.wait_ns = wait_ns;
-    attn_fwd_tc<FWD_FULL><<<dim3(n_tiles, s.Hq / 2, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp); count_launch();
+    attn_fwd_tc<FWD_FULL><<<tile_grid(s.Hq / 2, n_tiles, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp); count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || scores == nullptr) return e;
     ScParams sp{s.Lq, s.Lkv, s.Hq, s.Hkv, s.G(), row_begin, row_begin + row_count, row_count,
@@ -779,7 +779,7 @@ cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
             sp.tma_store = 1;
     }
-    attn_scores_tc<<<dim3(n_tiles, s.Hkv, s.B), SC_THREADS, kScSmem, st>>>(mq, mk, ms, sp); count_launch();
+    attn_scores_tc<<<tile_grid(s.Hkv, n_tiles, s.B), SC_THREADS, kScSmem, st>>>(mq, mk, ms, sp); count_launch();
     return cudaGetLastError();
 }
 
@@ -813,10 +813,10 @@ cudaError_t sparse_pair_tc_launch(const Shape &s, const void *q, const void *k, 
     fp.window = window; fp.W = W; fp.selmask = mask; fp.wl = wl; fp.gate = gate;
     fp.out_g = (__nv_bfloat16 *)og; fp.out_l = (__nv_bfloat16 *)ol;
     const int n_tiles = (s.Lq + BM - 1) / BM;
-    attn_fwd_tc<FWD_WIN><<<dim3(n_tiles, s.Hq / 2, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp); count_launch();
+    attn_fwd_tc<FWD_WIN><<<tile_grid(s.Hq / 2, n_tiles, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp); count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    attn_fwd_tc<FWD_SEL><<<dim3(n_tiles, s.Hq / 2, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp); count_launch();
+    attn_fwd_tc<FWD_SEL><<<tile_grid(s.Hq / 2, n_tiles, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp); count_launch();
     return cudaGetLastError();
 }
 

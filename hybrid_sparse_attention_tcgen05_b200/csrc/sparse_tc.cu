@@ -82,12 +82,12 @@ sparse_dense_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     SdBars *bars = reinterpret_cast<SdBars *>(smem + TILE + SD_KV * TILE);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tile = gridDim.x - 1 - blockIdx.x;
+    int tile, b;
+    tile_of_block((p.Lq + BM - 1) / BM, tile, b);   // heaviest row tiles first
     const int r0 = tile * BM;
     const int r_end = min(r0 + BM, p.Lq);
-    const int h = blockIdx.y;
+    const int h = blockIdx.x;
     const int g = h / p.G;
-    const int b = blockIdx.z;
     const int off = p.Lkv - p.Lq;
     const int pos_first = off + r0;
     const int pos_last = off + r_end - 1;
@@ -462,7 +462,7 @@ cudaError_t sparse_dense_tc_launch(const Shape &s, const void *q, const void *k,
     SdParams p{s.Lq, s.Lkv, s.Hq, s.Hkv, s.G(), window, W, s.scale * kLog2e, mask, gate,
                (__nv_bfloat16 *)out, (__nv_bfloat16 *)og, (__nv_bfloat16 *)ol, status, wait_ns};
     const int n_tiles = (s.Lq + BM - 1) / BM;
-    sparse_dense_tc<<<dim3(n_tiles, s.Hq, s.B), SD_THREADS, kSdSmem, st>>>(mq, mk, mv, p); count_launch();
+    sparse_dense_tc<<<tile_grid(s.Hq, n_tiles, s.B), SD_THREADS, kSdSmem, st>>>(mq, mk, mv, p); count_launch();
     return cudaGetLastError();
 }
 

@@ -89,6 +89,22 @@ __device__ __forceinline__ float ex2_mix(float x, int c) {
     return ex2(x);
 }
 
+// Row-tile grids are launched as (heads, row tiles x batch): the hardware
+// hands out blocks in linear order with x fastest, so the heaviest causal
+// row tile of every head and batch is dispatched before any lighter one.
+// When tiles x batch exceed the y limit the batch moves to z.
+inline dim3 tile_grid(int heads, int n_tiles, int batch) {
+    if ((long long)n_tiles * batch <= 65535) return dim3(heads, n_tiles * batch, 1);
+    return dim3(heads, n_tiles, batch);
+}
+
+// This block's row tile (0 = first 128 rows) and batch under tile_grid.
+__device__ __forceinline__ void tile_of_block(int n_tiles, int &tile, int &b) {
+    const int nb_y = gridDim.y / n_tiles;   // batches folded into y (1 when z carries them)
+    tile = n_tiles - 1 - (int)blockIdx.y / nb_y;
+    b = (int)blockIdx.z + (int)blockIdx.y % nb_y;
+}
+
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
