@@ -110,8 +110,9 @@ int run_full(const Shape &s, const void *q, const void *k, const void *v, void *
 }
 
 int run_topk(const Shape &s, const float *scores, long long ld, int row_begin, int row_count,
-             int topk, int32_t *idx, cudaStream_t st) {
-    return cuda_status(topk_launch(s, scores, ld, row_begin, row_count, topk, idx, st));
+             int topk, int32_t *idx, cudaStream_t st, uint32_t *mask = nullptr, bool *mask_done = nullptr) {
+    return cuda_status(topk_launch(s, scores, ld, row_begin, row_count, topk, idx, st, mask,
+                                   mask ? selmask_words(s) : 0, mask_done));
 }
 
 // Which sparse-layer kernel to run.  Both compute the same two softmaxes;
@@ -273,22 +274,26 @@ int hysparse_block(const hs_shape *shape, const void *q_full, const void *k, con
     float *lse_buf = lse ? lse : reinterpret_cast<float *>(w + L.block_lse);
     int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(w + L.block_idx);
     cudaStream_t st = (cudaStream_t)stream;
+    // the index set is shared by every sparse layer of the block, and so is
+    // the dense path's bitmask built from it: the top-k kernel writes it with
+    // the indices where it can, else one pass over the index lists builds it
+    const bool dense = n_sparse > 0 && prefer_dense_sparse(s, topk, window) && sparse_pair_supported(s);
+    uint32_t *mask = dense ? reinterpret_cast<uint32_t *>(w + ws_layout(s, topk, 1).selmask) : nullptr;
+    bool mask_all = dense;
     for (int r0 = 0; r0 < s.Lq; r0 += chunk) {
         const int rows = (s.Lq - r0 < chunk) ? s.Lq - r0 : chunk;
         rc = run_full(s, q_full, k, v, out_full, lse_buf, scores, s.Lkv, r0, rows, ws, st);
         if (rc != HS_OK) return rc;
-        rc = run_topk(s, scores, s.Lkv, r0, rows, topk, idx, st);
+        bool done = false;
+        rc = run_topk(s, scores, s.Lkv, r0, rows, topk, idx, st, mask, &done);
         if (rc != HS_OK) return rc;
+        mask_all = mask_all && done;
     }
-    // the index set is shared by every sparse layer of the block, and so is
-    // the dense path's bitmask built from it
-    bool mask_ready = false;
-    if (n_sparse > 0 && prefer_dense_sparse(s, topk, window) && sparse_pair_supported(s)) {
-        uint32_t *mask = reinterpret_cast<uint32_t *>(w + ws_layout(s, topk, 1).selmask);
+    if (dense && !mask_all) {
         rc = cuda_status(selmask_build_launch(s, idx, topk, mask, reinterpret_cast<unsigned int *>(ws), st));
         if (rc != HS_OK) return rc;
-        mask_ready = true;
     }
+    const bool mask_ready = dense;
     for (int n = 0; n < n_sparse; ++n) {
         rc = run_sparse(s, q_sparse[n], k, v, idx, topk, gate_logit[n], window, out_sparse[n],
                         nullptr, nullptr, ws, st, mask_ready);

@@ -80,7 +80,10 @@ cudaError_t sparse_pair_tc_launch(const Shape &s, const void *q, const void *k, 
 unsigned long long wait_limit_ns();
 
 // topk.cu
+// mask (optional, [B][Hkv][Lq][W] words): also write the rows' selection
+// bitmask; *mask_done tells whether every row of the launch got one.
 cudaError_t topk_launch(const Shape &s, const float *scores, long long ld, int row_begin,
-                        int row_count, int topk, int32_t *idx, cudaStream_t st);
+                        int row_count, int topk, int32_t *idx, cudaStream_t st, uint32_t *mask = nullptr,
+                        int W = 0, bool *mask_done = nullptr);
 
 }  // namespace hs

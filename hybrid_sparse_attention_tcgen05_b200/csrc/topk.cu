@@ -353,7 +353,8 @@ __device__ __forceinline__ unsigned int wk_find(const unsigned int *h, unsigned 
 template <bool AL>
 __global__ void __launch_bounds__(WK_WARPS * 32, 5)
 topk_warp_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv, int Hkv, int row_begin,
-                 int row_count, int topk, long long n_items, int32_t *__restrict__ idx) {
+                 int row_count, int topk, long long n_items, int32_t *__restrict__ idx, uint32_t *__restrict__ mask,
+                 int W) {
     __shared__ __align__(16) unsigned int hist_all[WK_WARPS][WK_BINS];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long item = (long long)blockIdx.x * WK_WARPS + warp;
@@ -365,8 +366,14 @@ topk_warp_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv
     const int n = Lkv - Lq + i + 1;
     const unsigned int *u = reinterpret_cast<const unsigned int *>(scores + ((size_t)bg * row_count + r) * ld);
     int32_t *o = idx + ((size_t)bg * Lq + i) * (size_t)topk;
+    uint32_t *mrow = mask ? mask + ((size_t)bg * Lq + i) * (size_t)W : nullptr;
     if (n <= topk) {
         for (int t = lane; t < topk; t += 32) o[t] = t < n ? t : -1;
+        if (mrow)
+            for (int w = lane; w < W; w += 32) {
+                const int lo = 32 * w;
+                mrow[w] = lo + 32 <= n ? FULL : (lo < n ? (1u << (n - lo)) - 1u : 0u);
+            }
         return;
     }
     unsigned int *h = hist_all[warp];
@@ -479,13 +486,27 @@ topk_warp_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv
             at += sel[c];
         }
         base += tot;
+        if (mrow) {
+            // bitmask: lanes 8m .. 8m+7 hold keys 32m' .. 32m'+31 of word m' =
+            // g0/8 + m; their 4-bit nibbles are OR-ed across the 8 lanes
+            unsigned int wd = ((sel[0] ? 1u : 0u) | (sel[1] ? 2u : 0u) | (sel[2] ? 4u : 0u) | (sel[3] ? 8u : 0u))
+                              << (4 * (lane & 7));
+            wd |= __shfl_xor_sync(FULL, wd, 1);
+            wd |= __shfl_xor_sync(FULL, wd, 2);
+            wd |= __shfl_xor_sync(FULL, wd, 4);
+            const int w = g0 / 8 + (lane >> 3);
+            if ((lane & 7) == 0 && w < W) mrow[w] = wd;
+        }
     }
+    if (mrow)   // words past the row's causal end
+        for (int w = 4 * ((n4 + 32) / 32) + lane; w < W; w += 32) mrow[w] = 0u;
 }
 
 }  // namespace
 
 cudaError_t topk_launch(const Shape &s, const float *scores, long long ld, int row_begin, int row_count,
-                        int topk, int32_t *idx, cudaStream_t st) {
+                        int topk, int32_t *idx, cudaStream_t st, uint32_t *mask, int W, bool *mask_done) {
+    if (mask_done) *mask_done = false;
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -494,28 +515,28 @@ cudaError_t topk_launch(const Shape &s, const float *scores, long long ld, int r
         attr = true;
     }
     const long long n_items = (long long)s.B * s.Hkv * row_count;
+    const long long off = (long long)s.Lkv - s.Lq;
+    const bool al = (reinterpret_cast<uintptr_t>(scores) & 15u) == 0 && (ld & 3) == 0;
     // HYSPARSE_TOPK_PATH=warp|block forces one kernel (the tests run both)
     const char *force = getenv("HYSPARSE_TOPK_PATH");
-    const bool use_warp = force && strcmp(force, "warp") == 0    ? true
-                          : force && strcmp(force, "block") == 0 ? false
-                                                                 : n_items >= kWarpMinItems;
-    if (use_warp) {
-        const bool al = (reinterpret_cast<uintptr_t>(scores) & 15u) == 0 && (ld & 3) == 0;
+    const bool f_warp = force && strcmp(force, "warp") == 0, f_block = force && strcmp(force, "block") == 0;
+    const bool many = f_warp || (!f_block && n_items >= kWarpMinItems);
+    if (many) {
         const unsigned int grid = (unsigned int)((n_items + WK_WARPS - 1) / WK_WARPS);
         if (al)
             topk_warp_kernel<true><<<grid, WK_WARPS * 32, 0, st>>>(scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin,
-                                                                   row_count, topk, n_items, idx);
+                                                                   row_count, topk, n_items, idx, mask, W);
         else
             topk_warp_kernel<false><<<grid, WK_WARPS * 32, 0, st>>>(scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin,
-                                                                    row_count, topk, n_items, idx);
+                                                                    row_count, topk, n_items, idx, mask, W);
         count_launch();
+        if (mask_done) *mask_done = mask != nullptr;
         return cudaGetLastError();
     }
     // Few rows (decode): one CTA per row.  Rows are ordered by causal length
     // n = off + row_begin + r + 1: those with n <= kSmemKeys run with the row
     // cached in shared memory (sized for the longest of them), the rest read
     // global memory.
-    const long long off = (long long)s.Lkv - s.Lq;
     const long long split = max(0ll, min((long long)row_count, (long long)kSmemKeys - off - row_begin));
     if (split > 0) {
         const long long n_max = off + row_begin + split;

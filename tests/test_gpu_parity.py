@@ -176,6 +176,28 @@ def test_topk_synthetic_rows_bit_exact(case, kernel, monkeypatch):
     assert torch.equal(idx.cpu(), o_idx)
 
 
+@pytest.mark.parametrize("topk_path", ["warp", "block"])
+@pytest.mark.parametrize("Lkv", [1000, 8500])
+def test_block_selection_mask_matches_stages(topk_path, Lkv, monkeypatch):
+    """hysparse_block on the dense sparse path: with the one-warp-per-row
+    top-k kernel the bitmask comes from the top-k pass itself, with the
+    one-CTA-per-row kernel from a pass over the index lists; either way the
+    outputs equal the stage calls' (whose sparse_attn builds the bitmask from
+    the index lists)."""
+    monkeypatch.setenv("HYSPARSE_SPARSE_PATH", "dense")
+    monkeypatch.setenv("HYSPARSE_TOPK_PATH", topk_path)
+    Lq = 1000 if Lkv == 1000 else 600     # the 8500 case: a row longer than 8192 keys
+    w = gen.Workload("bf16_mask_block", 1, Lq, Lkv, 8, 2, 128, "bf16", 100, 64, 2, "shifted")
+    inp = gen.make_inputs(w, seed=3, device=DEV)
+    out, lse, idx, _, outs = run_stages(inp, w)
+    of, lb, ib, ob = hs.block(inp["q"], inp["k"], inp["v"], inp["q_sparse"], inp["gate"], w.topk, w.window)
+    torch.cuda.synchronize()
+    assert torch.equal(ib, idx)
+    assert torch.equal(of, out)
+    for n in range(w.n_sparse):
+        assert torch.equal(ob[n], outs[n][0])
+
+
 # ------------------------------------------------------------- shape sweep
 
 SWEEP = [
