@@ -89,7 +89,7 @@ struct FwdParams {
     // sparse-layer modes
     int window, W;                   // window length; words per selection-mask row
     const uint32_t *selmask;         // [B][Hkv][Lq][W]
-    float *wl;                       // [B][Lq][Hq][128] window branch, normalised (fp32)
+    uint32_t *wl;                    // [B][Lq][Hq][128] window branch, normalised, bf16 pairs
     const float *gate;               // [B][Lq][Hq]
     __nv_bfloat16 *out_g, *out_l;    // optional branch outputs
 };
@@ -397,11 +397,12 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             }
         }
         if (fin && MODE == FWD_WIN) {
-            // normalised window branch, fp32, for the select pass to merge
+            // normalised window branch, bf16 (the precision of the branch
+            // output), for the select pass to merge
             tc_fence_after();
             const int h = h0 + w;
             const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-            float4 *wrow = reinterpret_cast<float4 *>(p.wl + (((size_t)b * p.Lq + row) * p.Hq + h) * HD);
+            uint4 *wrow = reinterpret_cast<uint4 *>(p.wl + (((size_t)b * p.Lq + row) * p.Hq + h) * (HD / 2));
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
@@ -409,9 +410,12 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                 tmem_wait_ld();
                 if (valid) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        wrow[8 * c + e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
-                                                      __uint_as_float(o[4 * e + 2]) * inv_l, __uint_as_float(o[4 * e + 3]) * inv_l);
+                    for (int e = 0; e < 4; ++e)
+                        wrow[4 * c + e] = make_uint4(
+                            pack_bf16(__uint_as_float(o[8 * e]) * inv_l, __uint_as_float(o[8 * e + 1]) * inv_l),
+                            pack_bf16(__uint_as_float(o[8 * e + 2]) * inv_l, __uint_as_float(o[8 * e + 3]) * inv_l),
+                            pack_bf16(__uint_as_float(o[8 * e + 4]) * inv_l, __uint_as_float(o[8 * e + 5]) * inv_l),
+                            pack_bf16(__uint_as_float(o[8 * e + 6]) * inv_l, __uint_as_float(o[8 * e + 7]) * inv_l));
                 }
             }
         }
@@ -423,7 +427,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             const size_t ro = ((size_t)b * p.Lq + row) * p.Hq + h;
             float sg = 0.f;
             if (valid) sg = 1.0f / (1.0f + expf(-p.gate[ro]));
-            const float4 *wrow = reinterpret_cast<const float4 *>(p.wl + ro * HD);
+            const uint4 *wrow = reinterpret_cast<const uint4 *>(p.wl + ro * (HD / 2));
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
@@ -431,17 +435,25 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                 tmem_wait_ld();
                 if (valid) {
                     uint32_t po[16], pg[16], pl[16];
+                    uint32_t wq[16];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint4 t4 = wrow[4 * c + e];
+                        wq[4 * e] = t4.x; wq[4 * e + 1] = t4.y; wq[4 * e + 2] = t4.z; wq[4 * e + 3] = t4.w;
+                    }
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float4 wv = wrow[8 * c + e];
+                        const float4 wv = make_float4(__uint_as_float(wq[2 * e] << 16), __uint_as_float(wq[2 * e] & 0xffff0000u),
+                                                      __uint_as_float(wq[2 * e + 1] << 16),
+                                                      __uint_as_float(wq[2 * e + 1] & 0xffff0000u));
                         const float g0 = __uint_as_float(o[4 * e]) * inv_l, g1 = __uint_as_float(o[4 * e + 1]) * inv_l;
                         const float g2 = __uint_as_float(o[4 * e + 2]) * inv_l, g3 = __uint_as_float(o[4 * e + 3]) * inv_l;
                         po[2 * e] = pack_bf16(sg * g0 + (1.f - sg) * wv.x, sg * g1 + (1.f - sg) * wv.y);
                         po[2 * e + 1] = pack_bf16(sg * g2 + (1.f - sg) * wv.z, sg * g3 + (1.f - sg) * wv.w);
                         pg[2 * e] = pack_bf16(g0, g1);
                         pg[2 * e + 1] = pack_bf16(g2, g3);
-                        pl[2 * e] = pack_bf16(wv.x, wv.y);
-                        pl[2 * e + 1] = pack_bf16(wv.z, wv.w);
+                        pl[2 * e] = wq[2 * e];
+                        pl[2 * e + 1] = wq[2 * e + 1];
                     }
                     uint4 *d0 = reinterpret_cast<uint4 *>(p.out + ro * HD + 32 * c);
 #pragma unroll
@@ -787,11 +799,11 @@ bool sparse_pair_supported(const Shape &s) {
     return s.dtype == HS_BF16 && s.d == 128 && (s.G() % 2) == 0 && s.Lq >= 64;
 }
 
-size_t sparse_pair_wl_bytes(const Shape &s) { return (size_t)s.B * s.Lq * s.Hq * 128 * sizeof(float); }
+size_t sparse_pair_wl_bytes(const Shape &s) { return (size_t)s.B * s.Lq * s.Hq * 128 * sizeof(uint16_t); }
 
 cudaError_t sparse_pair_tc_launch(const Shape &s, const void *q, const void *k, const void *v, const float *gate,
                                   int window, void *out, void *og, void *ol, const uint32_t *mask, int W,
-                                  float *wl, unsigned int *status, unsigned long long wait_ns, cudaStream_t st) {
+                                  uint32_t *wl, unsigned int *status, unsigned long long wait_ns, cudaStream_t st) {
     using namespace tc;
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, s.Hq, s.Lq, s.B) || !make_map(&mk, k, s.Hkv, s.Lkv, s.B) ||

@@ -157,7 +157,7 @@ int run_sparse(const Shape &s, const void *q, const void *k, const void *v, cons
         const WsLayout L = ws_layout(s, topk, 1);
         uint32_t *mask = reinterpret_cast<uint32_t *>(reinterpret_cast<char *>(ws) + L.selmask);
         if (sparse_pair_supported(s)) {
-            float *wl = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + L.wl);
+            uint32_t *wl = reinterpret_cast<uint32_t *>(reinterpret_cast<char *>(ws) + L.wl);
             cudaError_t e = mask_ready ? cudaSuccess : selmask_build_launch(s, idx, topk, mask, status, st);
             if (e == cudaSuccess)
                 e = sparse_pair_tc_launch(s, q, k, v, gate, window, out, og, ol, mask, selmask_words(s), wl, status,

@@ -67,13 +67,13 @@ cudaError_t selmask_build_launch(const Shape &s, const int32_t *idx, int topk, u
                                  cudaStream_t st);
 
 // attn_tc.cu, dense-masked sparse layer on the paired-head pipeline of the
-// full layer (even G): window branch into `wl` (fp32), then the masked global
+// full layer (even G): window branch into `wl` (bf16), then the masked global
 // branch merged by the gate.
 bool sparse_pair_supported(const Shape &s);
 size_t sparse_pair_wl_bytes(const Shape &s);
 cudaError_t sparse_pair_tc_launch(const Shape &s, const void *q, const void *k, const void *v, const float *gate,
                                   int window, void *out, void *og, void *ol, const uint32_t *mask, int W,
-                                  float *wl, unsigned int *status, unsigned long long wait_ns, cudaStream_t st);
+                                  uint32_t *wl, unsigned int *status, unsigned long long wait_ns, cudaStream_t st);
 
 // Upper bound (ns) on any single barrier wait inside a kernel; after it the
 // kernel records HS_ERR_TIMEOUT in the workspace status word and returns.
