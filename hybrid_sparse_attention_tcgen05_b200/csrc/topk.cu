@@ -378,22 +378,77 @@ topk_warp_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv
     }
     unsigned int *h = hist_all[warp];
     wk_zero(h, lane);
+    __syncwarp();
 
     const int n4 = n >> 2, nt = n - 4 * n4;
     const unsigned int xt = lane < nt ? __ldg(u + 4 * n4 + lane) : 0u;   // tail keys (< 4)
-    unsigned int mx = lane < nt ? xt : 0u, mn = lane < nt ? xt : FULL;
-    for (int g = lane; g < n4; g += 32) {
-        const uint4 v = ld4<AL>(u, g);
-        mx = max(mx, max(max(v.x, v.y), max(v.z, v.w)));
-        mn = min(mn, min(min(v.x, v.y), min(v.z, v.w)));
+    unsigned int M = 0u, pre = 0u, remaining = (unsigned int)topk, cnt_eq = (unsigned int)n;
+    int hs_ = 32, top = -1;
+    if (n >= 1024) {
+        // First digit without a separate max / min pass: the digit range comes
+        // from 8 sampled 32-key lines (keys outside it are clamped into the
+        // edge bins) while the same pass takes the row's exact max and min.
+        // Only if the k-th key falls in a clamped edge bin is the pass redone
+        // over the exact range.
+        unsigned int xs[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) xs[q] = __ldg(u + (int)(((long long)(n - 32) * q) / 7) + lane);
+        unsigned int smx = xs[0], smn = xs[0];
+#pragma unroll
+        for (int q = 1; q < 8; ++q) {
+            smx = max(smx, xs[q]);
+            smn = min(smn, xs[q]);
+        }
+        const unsigned int Ms = __reduce_max_sync(FULL, smx), ms = __reduce_min_sync(FULL, smn);
+        if (Ms > ms) {
+            const int tp = 32 - __clz(Ms - ms), s = max(0, tp - WK_BITS);
+            const unsigned int nbm1 = (1u << (tp - s)) - 1u;
+            unsigned int mx = lane < nt ? xt : 0u, mn = lane < nt ? xt : FULL;
+            auto bin = [&](unsigned int x) { return x > Ms ? 0u : min(nbm1, (Ms - x) >> s); };
+            for (int g = lane; g < n4; g += 32) {
+                const uint4 v = ld4<AL>(u, g);
+                mx = max(mx, max(max(v.x, v.y), max(v.z, v.w)));
+                mn = min(mn, min(min(v.x, v.y), min(v.z, v.w)));
+                atomicAdd(&h[bin(v.x)], 1u);
+                atomicAdd(&h[bin(v.y)], 1u);
+                atomicAdd(&h[bin(v.z)], 1u);
+                atomicAdd(&h[bin(v.w)], 1u);
+            }
+            if (lane < nt) atomicAdd(&h[bin(xt)], 1u);
+            const unsigned int Mx = __reduce_max_sync(FULL, mx), Mn = __reduce_min_sync(FULL, mn);
+            __syncwarp();
+            unsigned int rem2, cnt;
+            const unsigned int dig = wk_find(h, remaining, lane, rem2, cnt);
+            __syncwarp();
+            wk_zero(h, lane);
+            __syncwarp();
+            const bool clamped = (dig == 0u && Mx > Ms) || (dig == nbm1 && ((Ms - Mn) >> s) > nbm1);
+            if (!clamped) {
+                M = Ms;
+                pre = dig;
+                remaining = rem2;
+                cnt_eq = cnt;
+                hs_ = s;
+                top = s;
+            } else {
+                M = Mx;
+                top = Mx > Mn ? 32 - __clz(Mx - Mn) : 0;
+            }
+        }
     }
-    const unsigned int M = __reduce_max_sync(FULL, mx);
-    const unsigned int range = M - __reduce_min_sync(FULL, mn);
-    const int L = range ? 32 - __clz(range) : 0;
-    __syncwarp();
+    if (top < 0) {   // short or constant-looking sample: exact max / min first
+        unsigned int mx = lane < nt ? xt : 0u, mn = lane < nt ? xt : FULL;
+        for (int g = lane; g < n4; g += 32) {
+            const uint4 v = ld4<AL>(u, g);
+            mx = max(mx, max(max(v.x, v.y), max(v.z, v.w)));
+            mn = min(mn, min(min(v.x, v.y), min(v.z, v.w)));
+        }
+        M = __reduce_max_sync(FULL, mx);
+        const unsigned int range = M - __reduce_min_sync(FULL, mn);
+        top = range ? 32 - __clz(range) : 0;
+        __syncwarp();
+    }
 
-    unsigned int pre = 0u, remaining = (unsigned int)topk, cnt_eq = (unsigned int)n;
-    int hs_ = 32, top = L;
     while (top > 0) {
         const int s = max(0, top - WK_BITS);
         const unsigned int msk = (1u << (top - s)) - 1u;
