@@ -416,7 +416,7 @@ def bench_ours(args, w, ws_, rank, local):
         peak = peaks["bf16_tflops"]
         roof = {"kernel": "full_attn_scores", "bound": "tensor", "unit": "TFLOP/s",
                 "work": "6*d*Hq per causal pair (QK^T+PV forward, QK^T score pass)"}
-        key, srcs = "full_attn_scores", ("attn_tc.cu",)
+        key, srcs = "full_attn_scores", ("attn_tc.cu", "tc_attn.cuh", "tc_util.cuh")
     elif dom == "topk":
         launches = n_chunks
         dur_s = per["topk"] / launches / 1e3
@@ -437,7 +437,7 @@ def bench_ours(args, w, ws_, rank, local):
                 "bound": "tensor", "unit": "TFLOP/s",
                 "work": "4*d*Hq*(k_eff + w_eff) per row: the FLOPs the method needs",
                 "executed_tflops": wm["flops_full_fwd"] / dur_s / 1e12}
-        key, srcs = "sparse_pair", ("attn_tc.cu", "sparse_tc.cu")
+        key, srcs = "sparse_pair", ("attn_tc.cu", "sparse_tc.cu", "tc_attn.cuh", "tc_util.cuh")
     else:
         launches = w.n_sparse
         dur_s = per["sparse"] / launches / 1e3

@@ -22,6 +22,11 @@
 //   warp 8     TMA producer (Q tiles once, then K and V tiles through a
 //              3-slot ring filled in the order the MMAs consume them)
 //   warp 9     MMA issuer (one thread)
+//   warps 10-11 idle; they complete the third warpgroup so that warps 8-11
+//              can hand registers to the softmax warpgroups (setmaxnreg:
+//              168 per thread at launch, then 104 for warps 8-11 and 200
+//              for warps 0-7, which holds a row of S and its packed
+//              f32x2 arithmetic without spills)
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 f32 columns each.  P (bf16) goes
 // to shared memory in the swizzled layout of a Q tile, so the softmax
 // threads release S_j as soon as they have read it and S_{j+1} = Q K_{j+1}^T
@@ -162,8 +167,9 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
     volatile int *abort = &bars->abort;
-
-    if (warp == 8) {
+    if (warp >= 8) {
+      regs_release<kFwdCtlRegs>();
+      if (warp == 8) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch(&tq);
@@ -196,7 +202,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                     mbar_drain(smem_u32(&bars->kv_full[it % FWD_KV]), (it / FWD_KV) & 1);
             }
         }
-    } else if (warp == 9) {
+      } else if (warp == 9) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t tS[2] = {tmem, tmem + 128}, tO[2] = {tmem + 256, tmem + 384};
@@ -240,7 +246,9 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             mma_commit(smem_u32(&bars->drain));
             mbar_drain(smem_u32(&bars->drain), 0);
         }
+      }
     } else {
+        regs_acquire<kFwdSoftRegs>();
         // ------------------------------------------------ softmax warpgroups
         const int w = warp >> 2;
         const int tw = threadIdx.x - 128 * w;
@@ -300,13 +308,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                     if (j0 + c > pos) s[c] = -INFINITY;
             }
             float m4[4] = {s[0], s[1], s[2], s[3]};
-            if (MODE == FWD_FULL) {
 #pragma unroll
-                for (int c = 4; c < 128; c += 2) m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], s[c], s[c + 1]);
-            } else {   // measured: the two-input chain is faster in the masked modes
-#pragma unroll
-                for (int c = 4; c < 128; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
-            }
+            for (int c = 4; c < 128; c += 2) m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], s[c], s[c + 1]);
             const float mx2 = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c2;
             // PV of the previous tile done: O is stable and the P buffer is free
             if (j > 0) {
@@ -343,16 +346,9 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int c = ch * 8 + 2 * e;
-                    float2 ab;
-                    if (MODE != FWD_FULL) {   // measured: packed pairs spill or lose in the masked modes
-                        ab = make_float2(ex2_mix<kFwdPolyEvery>(fmaf(s[c], c2, -mref), c),
-                                         ex2_mix<kFwdPolyEvery>(fmaf(s[c + 1], c2, -mref), c + 1));
-                        if (e & 1) { ps23.x += ab.x; ps23.y += ab.y; } else { ps01.x += ab.x; ps01.y += ab.y; }
-                    } else {
-                        const float2 t = ffma2(make_float2(s[c], s[c + 1]), c2v, mv);
-                        ab = make_float2(ex2_mix<kFwdPolyEvery>(t.x, c), ex2_mix<kFwdPolyEvery>(t.y, c + 1));
-                        if (e & 1) ps23 = fadd2(ps23, ab); else ps01 = fadd2(ps01, ab);
-                    }
+                    const float2 t = ffma2(make_float2(s[c], s[c + 1]), c2v, mv);
+                    const float2 ab = make_float2(ex2_mix<kFwdPolyEvery>(t.x, c), ex2_mix<kFwdPolyEvery>(t.y, c + 1));
+                    if (e & 1) ps23 = fadd2(ps23, ab); else ps01 = fadd2(ps01, ab);
                     pk[e] = pack_bf16(ab.x, ab.y);
                 }
                 const int half = ch >> 3, c8 = ch & 7;
@@ -747,6 +743,21 @@ bool full_attn_tc_supported(const Shape &s) {
     return s.dtype == HS_BF16 && s.d == 128 && (s.G() % 2) == 0 && s.Lkv < (1 << 24);
 }
 
+// One-time set-up of a forward instantiation: its dynamic shared memory, and
+// a check that it is launched with exactly the registers per thread that the
+// in-kernel hand-over between warpgroups is sized for (with fewer, the
+// softmax warpgroups' increase could never be satisfied).
+template <int MODE>
+static cudaError_t fwd_prepare() {
+    using namespace tc;
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdSmem);
+    if (e != cudaSuccess) return e;
+    cudaFuncAttributes a;
+    e = cudaFuncGetAttributes(&a, attn_fwd_tc<MODE>);
+    if (e != cudaSuccess) return e;
+    return a.numRegs == kFwdLaunchRegs ? cudaSuccess : cudaErrorInvalidDeviceFunction;
+}
+
 cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void *k, const void *v,
                                        void *out, float *lse, float *scores, long long ld,
                                        int row_begin, int row_count, float2 *stats,
@@ -759,7 +770,7 @@ cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void
         return cudaErrorInvalidValue;
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc<FWD_FULL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdSmem);
+        cudaError_t e = fwd_prepare<FWD_FULL>();
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(attn_scores_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScSmem);
         if (e != cudaSuccess) return e;
@@ -811,9 +822,9 @@ cudaError_t sparse_pair_tc_launch(const Shape &s, const void *q, const void *k, 
         return cudaErrorInvalidValue;
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc<FWD_WIN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdSmem);
+        cudaError_t e = fwd_prepare<FWD_WIN>();
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(attn_fwd_tc<FWD_SEL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdSmem);
+        e = fwd_prepare<FWD_SEL>();
         if (e != cudaSuccess) return e;
         attr_done = true;
     }

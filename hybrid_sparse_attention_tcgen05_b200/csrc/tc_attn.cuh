@@ -18,8 +18,31 @@ constexpr int HD = 128;                 // head dim
 constexpr int TILE = BM * HD * 2;       // one 128x128 bf16 tile: 32 KB
 constexpr int HALF = TILE / 2;          // one 64-column swizzled half: 16 KB
 constexpr int KV_STAGES = 4;
-constexpr int FWD_THREADS = 320;
+// Forward kernels: softmax warpgroups 0 and 1 (one query head each), then a
+// third warpgroup whose warp 8 issues the TMA loads and warp 9 the MMAs
+// (warps 10 and 11 only complete the warpgroup for the register hand-over).
+constexpr int FWD_THREADS = 384;
+// Registers per thread at launch (65536 / 384, rounded down to a multiple of
+// 8) and after the hand-over: the control warpgroup drops to kFwdCtlRegs and
+// the softmax warpgroups rise to kFwdSoftRegs.  The shares must add up to at
+// most what the block was launched with, or the increase never completes.
+constexpr int kFwdLaunchRegs = 168;
+constexpr int kFwdCtlRegs = 104;
+constexpr int kFwdSoftRegs = 200;
+static_assert(128 * kFwdCtlRegs + 256 * kFwdSoftRegs <= FWD_THREADS * kFwdLaunchRegs, "register hand-over over budget");
+static_assert(kFwdLaunchRegs * FWD_THREADS <= 65536, "launch registers");
 constexpr uint64_t kDrainNs = 1000000000ull;
+
+// Register hand-over between warpgroups (sm_100a setmaxnreg): every warp of
+// the warpgroup executes the same instruction.
+template <int N>
+__device__ __forceinline__ void regs_release() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_acquire() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
 
 __device__ __forceinline__ float ex2(float x) {
     float y;
