@@ -130,7 +130,8 @@ TOPK_BUCKET_EDGES = (9984, 25600)
 
 
 @pytest.mark.parametrize("case", ["ties", "ties_unaligned", "all_equal", "zeros_and_denormals", "long_rows",
-                                  "flat_narrow", "flat_long_unaligned", "many_rows_ties"]
+                                  "flat_narrow", "flat_long_unaligned", "many_rows_ties",
+                                  "many_rows_ties_aligned", "rows_8192", "short_rows_between_long"]
                          + [f"edge{e}" for e in TOPK_BUCKET_EDGES]
                          + [f"edge{e}_unaligned" for e in TOPK_BUCKET_EDGES])
 @pytest.mark.parametrize("kernel", ["block", "warp"])
@@ -154,10 +155,16 @@ def test_topk_synthetic_rows_bit_exact(case, kernel, monkeypatch):
         Lkv = 301
     elif case == "many_rows_ties":   # enough rows for the one-warp-per-row kernel by default
         B, Hkv, Lq, Lkv, k = 1, 2, 2100, 2203, 150
+    elif case == "many_rows_ties_aligned":   # 16-byte aligned rows, many per launch
+        B, Hkv, Lq, Lkv, k = 1, 2, 2100, 2204, 150
+    elif case == "rows_8192":        # the prefill8k row lengths at their longest
+        B, Hkv, Lq, Lkv, k = 1, 2, 300, 8192, 1000
+    elif case == "short_rows_between_long":   # rows with n <= k end every (b, g) block
+        B, Hkv, Lq, Lkv, k = 2, 2, 1500, 1500, 700
     s = torch.rand(B, Hkv, Lq, Lkv, generator=g)
     if case in ("ties", "ties_unaligned"):
         s = torch.round(s * 16) / 16
-    elif case == "many_rows_ties":
+    elif case.startswith("many_rows_ties") or case in ("rows_8192", "short_rows_between_long"):
         s = torch.round(s * 512) / 512
     elif case == "all_equal":
         s[:] = 0.125
@@ -250,6 +257,40 @@ def test_shape_sweep_all_rows(case, sparse_path):
     out, lse, idx, sc, outs = run_stages(inp, w, row_chunk=max(1, Lq // 3))
     rows = rows_for(B, Lq, range(Lq))
     oracle_check_rows(inp, w, rows, out, lse, idx, sc, outs)
+
+
+@pytest.mark.parametrize("sparse_path", ["dense", "gather"], indirect=True)
+def test_global_branch_far_below_unselected_keys(sparse_path):
+    """Unselected keys whose logits sit ~200 (log2 units) above every selected
+    key: a softmax reference taken over all keys would underflow every
+    selected term to zero.  Both sparse kernels take the reference over the
+    selected keys only and must give the exact global branch."""
+    B, L, Hq, Hkv, d, topk, window = 1, 640, 8, 2, 128, 48, 32
+    g = torch.Generator().manual_seed(11)
+    k = torch.randn(B, L, Hkv, d, generator=g) / d ** 0.5
+    v = torch.randn(B, L, Hkv, d, generator=g)
+    qs = torch.randn(B, L, Hq, d, generator=g) / d ** 0.5
+    trap = torch.arange(L) % 9 == 4                 # never selected, huge logits
+    k[:, trap] = 0.0
+    k[:, trap, :, 0] = 40.0
+    qs[..., 0] = 40.0                               # q'.k = 1600 on trap keys
+    gate = torch.randn(B, L, Hq, generator=g)
+    idx = torch.full((B, Hkv, L, topk), -1, dtype=torch.int32)
+    for gi in range(Hkv):
+        for i in range(L):
+            cand = torch.nonzero(~trap[: i + 1]).flatten()
+            pick = cand[torch.randperm(len(cand), generator=g)[:topk]].sort().values
+            idx[0, gi, i, : len(pick)] = pick.to(torch.int32)
+    k, v, qs = (t.to(torch.bfloat16) for t in (k, v, qs))
+    out, og, ol = hs.sparse_attn(qs.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), gate.to(DEV), window,
+                                 want_branches=True)
+    torch.cuda.synchronize()
+    rows = rows_for(B, L, range(L))
+    r_out, r_og, r_ol = oracle.sparse_rows(gather_rows(qs, rows), k, v, rows, L, scale_of(d),
+                                           gather_idx_rows(idx, rows), gather_rows(gate, rows), window)
+    check_out("global branch", gather_rows(og, rows), r_og, "bf16")
+    check_out("local branch", gather_rows(ol, rows), r_ol, "bf16")
+    check_out("out", gather_rows(out, rows), r_out, "bf16")
 
 
 # ------------------------------------------------- full-size, sampled rows
