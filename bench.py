@@ -379,7 +379,12 @@ def bench_ours(args, w, ws_, rank, local):
                 a_.copy_(b_, non_blocking=True)
             out_done[i_].record(s_out)
 
-    e2e_steps = max(4, min(args.steps, 8))
+    # enough steps that the pipeline's fill and drain (the first copy in
+    # before any compute, the last compute and copy out after the last copy
+    # in) are a small share of the timed region: about 1.5 s of device time,
+    # 4 to 32 steps (ms_per_step is already the max over ranks, so every rank
+    # runs the same count)
+    e2e_steps = int(max(4, min(32, 1500.0 / max(ms_per_step, 1e-3))))
     e2e_step(0)
     e2e_step(1)
     torch.cuda.synchronize()
