@@ -145,8 +145,9 @@ def source_hash(*names):
 
 def read_traffic(kernel_key: str, src_hash: str):
     """DRAM bytes per launch recorded from an ncu capture in
-    profiles/traffic.txt ("<key> <source-hash> <bytes-per-launch>"); None if
-    absent or taken on another version of the kernel source."""
+    profiles/traffic.txt ("<workload>/<kernel> <source-hash> <bytes-per-launch>");
+    None if absent, taken on another workload size or taken on another version
+    of the kernel source."""
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
@@ -453,7 +454,7 @@ def bench_ours(args, w, ws_, rank, local):
         key, srcs = "sparse_attn", ("sparse_mma.cu",)
     roof.update({"achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} (burst)",
                  "frac": achieved / peak, "launch_ms": dur_s * 1e3,
-                 "traffic": read_traffic(key, source_hash(*srcs))})
+                 "traffic": read_traffic(f"{w.name}/{key}", source_hash(*srcs))})
     stage_ctx = {
         "full": {"ms": per["full"], "tflops": (wm["flops_full_scores"] / (per["full"] / 1e3) / 1e12) if w.Lq > 1 else None,
                  "hbm_gbs": (wm["kv_bytes"] / (per["full"] / 1e3) / 1e9) if w.Lq == 1 else None},
