@@ -324,6 +324,22 @@ def bench_ours(args, w, ws_, rank, local):
         for name, e in seq:
             stage_ms[name] += prev.elapsed_time(e)
             prev = e
+    # the full layer's forward alone (S1: no score pass), for its own tensor
+    # rate beside the S1+S2 figure of the full stage (prefill only)
+    fwd_ms = None
+    if w.Lq > 1:
+        fwd_ms = 0.0
+        for _ in range(args.steps):
+            flush.fill_(1.0)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for c in range(n_chunks):
+                hs.full_attn_scores(q, k, v, want_scores=False, row_begin=c * chunk,
+                                    row_count=min(chunk, w.Lq - c * chunk), out=out, lse=lse, ws=ws_full)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            fwd_ms += e0.elapsed_time(e1) / args.steps
 
     # ---- end to end through the public API with host buffers
     # Each step copies its inputs from pinned host memory, runs the block and
@@ -457,7 +473,13 @@ def bench_ours(args, w, ws_, rank, local):
                  "traffic": read_traffic(f"{w.name}/{key}", source_hash(*srcs))})
     stage_ctx = {
         "full": {"ms": per["full"], "tflops": (wm["flops_full_scores"] / (per["full"] / 1e3) / 1e12) if w.Lq > 1 else None,
+                 "frac_of_peak": (wm["flops_full_scores"] / (per["full"] / 1e3) / 1e12 / peaks["bf16_tflops"])
+                 if w.Lq > 1 else None,
+                 "work": "6*d*Hq per causal pair (forward QK^T + PV, score-pass QK^T)" if w.Lq > 1 else None,
                  "hbm_gbs": (wm["kv_bytes"] / (per["full"] / 1e3) / 1e9) if w.Lq == 1 else None},
+        "full_forward_only": ({"ms": fwd_ms, "tflops": wm["flops_full_fwd"] / (fwd_ms / 1e3) / 1e12,
+                               "frac_of_peak": wm["flops_full_fwd"] / (fwd_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                               "work": "4*d*Hq per causal pair (QK^T + PV)"} if fwd_ms else None),
         "topk": {"ms": per["topk"], "gbs": (wm["score_bytes"] / 2 + 4.0 * w.B * w.Hkv * w.Lq * w.topk)
                  / (per["topk"] / 1e3) / 1e9},
         "sparse_per_layer": {"ms": per["sparse"] / max(1, w.n_sparse),
