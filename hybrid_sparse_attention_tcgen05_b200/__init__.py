@@ -163,9 +163,14 @@ def block(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_sparse: Sequence[
           gate_logit: Sequence[torch.Tensor], k_top: int, window: int, *, row_chunk: int = 0,
           out_full: Optional[torch.Tensor] = None, out_sparse: Optional[List[torch.Tensor]] = None,
           idx: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-          ws: Optional[torch.Tensor] = None, scale: Optional[float] = None):
-    """One hybrid block.  Returns (out_full, lse, idx, [out_sparse_n])."""
-    dev = _need_cuda(q, k, v, out_full, idx, lse, ws, *q_sparse, *gate_logit, *(out_sparse or []))
+          ws: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+          kv_len: Optional[torch.Tensor] = None):
+    """One hybrid block.  Returns (out_full, lse, idx, [out_sparse_n]).
+
+    kv_len (int32 [B] on the device, decode only): sequence b's cache is the
+    first kv_len[b] rows of k[b] and v[b], its new query at position
+    kv_len[b] - 1 (hysparse_block_varlen)."""
+    dev = _need_cuda(q, k, v, out_full, idx, lse, ws, kv_len, *q_sparse, *gate_logit, *(out_sparse or []))
     s = shape_of(q, k, scale)
     n = len(q_sparse)
     if len(gate_logit) != n:
@@ -184,6 +189,16 @@ def block(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_sparse: Sequence[
     qa = PA(*[x.data_ptr() for x in q_sparse])
     ga = PA(*[x.data_ptr() for x in gate_logit])
     oa = PA(*[x.data_ptr() for x in out_sparse])
+    if kv_len is not None:
+        if kv_len.dtype != torch.int32 or kv_len.shape != (s.B,) or not kv_len.is_contiguous():
+            raise TypeError("kv_len must be a contiguous int32 tensor of shape [B]")
+        st = _lib.lib().hysparse_block_varlen(
+            ctypes.byref(s), _ptr(kv_len), _ptr(q), _ptr(k), _ptr(v), _ptr(out_full), _ptr(lse), n,
+            ctypes.cast(qa, ctypes.c_void_p), ctypes.cast(ga, ctypes.c_void_p),
+            ctypes.cast(oa, ctypes.c_void_p), int(k_top), int(window), _ptr(idx),
+            _ptr(ws), ws.numel(), _stream(dev))
+        _lib.check(st, "hysparse_block_varlen")
+        return out_full, lse, idx, out_sparse
     st = _lib.lib().hysparse_block(
         ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(out_full), _ptr(lse), n,
         ctypes.cast(qa, ctypes.c_void_p), ctypes.cast(ga, ctypes.c_void_p),

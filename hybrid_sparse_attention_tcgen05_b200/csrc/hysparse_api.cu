@@ -246,14 +246,21 @@ int hysparse_sparse_attn(const hs_shape *shape, const void *q, const void *k, co
                       (cudaStream_t)stream);
 }
 
-int hysparse_block(const hs_shape *shape, const void *q_full, const void *k, const void *v,
-                   void *out_full, float *lse, int n_sparse, const void *const *q_sparse,
-                   const float *const *gate_logit, void *const *out_sparse, int topk, int window,
-                   int32_t *idx_out, int row_chunk, void *ws, size_t ws_bytes,
-                   hs_stream_t stream) {
+namespace {
+// hysparse_block, and hysparse_block_varlen when kv_len is set
+int block_impl(const hs_shape *shape, const int32_t *kv_len, const void *q_full, const void *k, const void *v,
+               void *out_full, float *lse, int n_sparse, const void *const *q_sparse,
+               const float *const *gate_logit, void *const *out_sparse, int topk, int window,
+               int32_t *idx_out, int row_chunk, void *ws, size_t ws_bytes, hs_stream_t stream) {
     Shape s;
     int rc = resolve_shape(shape, &s);
     if (rc != HS_OK) return rc;
+    if (kv_len != nullptr) {
+        // caches of different lengths: the bf16 decode path only
+        if (s.Lq != 1 || !use_decode_path(s)) return HS_ERR_UNSUPPORTED;
+        if ((reinterpret_cast<uintptr_t>(kv_len) & 3u) != 0) return HS_ERR_INVALID_ARG;
+        s.kv_len = kv_len;
+    }
     if (topk < 1 || topk > kMaxTopk || window < 1 || window > kMaxWindow || n_sparse < 0)
         return HS_ERR_INVALID_ARG;
     if (n_sparse > 0 && (q_sparse == nullptr || gate_logit == nullptr || out_sparse == nullptr))
@@ -300,6 +307,25 @@ int hysparse_block(const hs_shape *shape, const void *q_full, const void *k, con
         if (rc != HS_OK) return rc;
     }
     return HS_OK;
+}
+}  // namespace
+
+int hysparse_block(const hs_shape *shape, const void *q_full, const void *k, const void *v,
+                   void *out_full, float *lse, int n_sparse, const void *const *q_sparse,
+                   const float *const *gate_logit, void *const *out_sparse, int topk, int window,
+                   int32_t *idx_out, int row_chunk, void *ws, size_t ws_bytes,
+                   hs_stream_t stream) {
+    return block_impl(shape, nullptr, q_full, k, v, out_full, lse, n_sparse, q_sparse, gate_logit, out_sparse,
+                      topk, window, idx_out, row_chunk, ws, ws_bytes, stream);
+}
+
+int hysparse_block_varlen(const hs_shape *shape, const int32_t *kv_len, const void *q_full, const void *k,
+                          const void *v, void *out_full, float *lse, int n_sparse, const void *const *q_sparse,
+                          const float *const *gate_logit, void *const *out_sparse, int topk, int window,
+                          int32_t *idx_out, void *ws, size_t ws_bytes, hs_stream_t stream) {
+    if (kv_len == nullptr) return HS_ERR_INVALID_ARG;
+    return block_impl(shape, kv_len, q_full, k, v, out_full, lse, n_sparse, q_sparse, gate_logit, out_sparse,
+                      topk, window, idx_out, 0, ws, ws_bytes, stream);
 }
 
 int hysparse_workspace_status(void *ws, hs_stream_t stream) {

@@ -18,6 +18,10 @@ struct Shape {
     int B, Lq, Lkv, Hq, Hkv, d;
     int dtype;
     float scale;
+    // decode over caches of different lengths: kv_len[b] (device, int32) is
+    // sequence b's cache length (its new token at position kv_len[b] - 1);
+    // NULL = every sequence has Lkv.  Only the bf16 decode path reads it.
+    const int32_t *kv_len = nullptr;
     int G() const { return Hq / Hkv; }
 };
 
@@ -82,6 +86,8 @@ unsigned long long wait_limit_ns();
 // topk.cu
 // mask (optional, [B][Hkv][Lq][W] words): also write the rows' selection
 // bitmask; *mask_done tells whether every row of the launch got one.
+// Row lengths follow s.kv_len when it is set (decode over caches of
+// different lengths).
 cudaError_t topk_launch(const Shape &s, const float *scores, long long ld, int row_begin,
                         int row_count, int topk, int32_t *idx, cudaStream_t st, uint32_t *mask = nullptr,
                         int W = 0, bool *mask_done = nullptr);

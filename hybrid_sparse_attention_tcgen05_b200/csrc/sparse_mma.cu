@@ -73,7 +73,20 @@ struct SpParams {
     float scale_log2;
     unsigned int *status;
     unsigned long long wait_ns;
+    const int32_t *kv_len;   // [B] cache lengths (decode over caches of different lengths) or NULL
 };
+
+// Cache length of sequence b: kv_len[b] when given (a value outside
+// [1, Lkv] is reported and clamped, so no read leaves the cache), else Lkv.
+__device__ __forceinline__ int seq_len(const SpParams &p, int b) {
+    if (p.kv_len == nullptr) return p.Lkv;
+    const int L = __ldg(p.kv_len + b);
+    if (L < 1 || L > p.Lkv) {
+        report(p.status, HS_ERR_INVALID_ARG);
+        return L < 1 ? 1 : p.Lkv;
+    }
+    return L;
+}
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
@@ -281,7 +294,7 @@ __global__ void __launch_bounds__(SW * 32, 1) sparse_attn_mma(const SpParams p) 
     const int b = (int)(head_batch % p.B);
     const int g = (int)(head_batch / p.B);
     const int G = p.G;
-    const int pos = p.Lkv - p.Lq + i;
+    const int pos = seq_len(p, b) - p.Lq + i;
     uint8_t *wbase = smem + warp * SpSmem<NB>::WARP_BYTES;
     uint8_t *qs = wbase + ST * STAGE_BYTES;
     // stage the group's query rows (zero rows pad the heads up to 8*NB)
@@ -406,8 +419,9 @@ __global__ void __launch_bounds__(SW * 32, 1) decode_full_mma(const DecParams dp
         for (int kp = 0; kp < 4; ++kp)
             ldsm_x4(smem_u32(qs + (8 * nb + (lane & 7)) * RS + (32 * kp + 8 * (lane >> 3)) * 2),
                     bq[nb][2 * kp][0], bq[nb][2 * kp][1], bq[nb][2 * kp + 1][0], bq[nb][2 * kp + 1][1]);
+    const int Lb = seq_len(p, b);
     const int lo = ch * kDecChunk;
-    const int hi = min(p.Lkv, lo + kDecChunk);
+    const int hi = min(Lb, lo + kDecChunk);
     WarpCtx w;
     w.p = &p;
     w.kb = p.k + ((size_t)b * p.Lkv * p.Hkv + g) * 128;
@@ -422,7 +436,8 @@ __global__ void __launch_bounds__(SW * 32, 1) decode_full_mma(const DecParams dp
     w.stash_ld = p.Lkv;
     w.G = G;
     Branch<NB> br;
-    run_branch<NB>(w, false, bq, br);
+    if (lo < hi) run_branch<NB>(w, false, bq, br);
+    else br.init();   // a chunk past this sequence's cache: an empty partial (m = -inf, l = 0, O = 0)
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
@@ -472,7 +487,8 @@ __global__ void __launch_bounds__(256) decode_combine(const DecParams dp, float 
     if (scores == nullptr) return;
     const float *st = dp.stash + qrow * (size_t)p.Lkv;
     float *srow = scores + ((size_t)b * p.Hkv + g) * ld_scores;
-    for (int j = threadIdx.x; j < p.Lkv; j += blockDim.x) {
+    const int Lb = seq_len(p, b);
+    for (int j = threadIdx.x; j < Lb; j += blockDim.x) {
         float sc = 0.f;
         for (int h = 0; h < G; ++h) sc = fmaf(ex2f(st[(size_t)h * p.Lkv + j] - s_m[h]), s_il[h], sc);
         srow[j] = sc;
@@ -525,7 +541,7 @@ cudaError_t sparse_attn_mma_launch(const Shape &s, const void *q, const void *k,
                                    cudaStream_t st) {
     tc::SpParams p{(const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, idx, gate,
                    (__nv_bfloat16 *)out, (__nv_bfloat16 *)og, (__nv_bfloat16 *)ol, s.B, s.Lq, s.Lkv, s.Hq,
-                   s.Hkv, s.G(), topk, window, s.scale * kLog2e, status, wait_ns};
+                   s.Hkv, s.G(), topk, window, s.scale * kLog2e, status, wait_ns, s.kv_len};
     return s.G() <= 8 ? tc::launch_nb<1>(p, st) : tc::launch_nb<2>(p, st);
 }
 
@@ -545,7 +561,7 @@ cudaError_t decode_full_mma_launch(const Shape &s, const void *q, const void *k,
     tc::DecParams dp;
     dp.sp = tc::SpParams{(const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, nullptr,
                          nullptr, (__nv_bfloat16 *)out, nullptr, nullptr, s.B, 1, s.Lkv, s.Hq, s.Hkv, s.G(),
-                         1, 1, s.scale * kLog2e, status, 0};
+                         1, 1, s.scale * kLog2e, status, 0, s.kv_len};
     dp.part_o = reinterpret_cast<float *>(w);
     w += align_up(rows * nchunk * 128 * sizeof(float), 256);
     dp.part_ml = reinterpret_cast<float2 *>(w);

@@ -43,6 +43,15 @@ constexpr int kSmemKeys = 9984;
 // per-row kernel; fewer, longer rows (decode) take one CTA per row.
 constexpr long long kWarpMinItems = 4096;
 
+// Keys of row i of batch b: the causal prefix of its cache, whose length is
+// kv_len[b] when given (clamped to [1, Lkv]; the decode kernels report values
+// outside it), else Lkv.
+__device__ __forceinline__ int row_keys(const int32_t *kv_len, int b, int Lq, int Lkv, int i) {
+    int L = Lkv;
+    if (kv_len != nullptr) L = min(max(__ldg(kv_len + b), 1), Lkv);
+    return L - Lq + i + 1;
+}
+
 struct TopkShared {
     unsigned int h[2][kBins];      // digit histograms (passes alternate)
     unsigned int wa[NW], wb[NW];   // per-warp partials
@@ -139,7 +148,7 @@ __device__ __forceinline__ void find_bin(TopkShared &sh, const unsigned int *his
 template <bool SMEM>
 __global__ void __launch_bounds__(NT, 4)
 topk_radix_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv, int Hkv, int row_begin,
-                  int row_count, int r_lo, int topk, int32_t *__restrict__ idx) {
+                  int row_count, int r_lo, int topk, int32_t *__restrict__ idx, const int32_t *__restrict__ kv_len) {
     extern __shared__ __align__(16) unsigned int row_cache[];
     __shared__ TopkShared sh;
     __shared__ int cnt_gt[NW], cnt_eq[NW];
@@ -147,7 +156,7 @@ topk_radix_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lk
     const int r = r_lo + blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int i = row_begin + r;
-    const int n = Lkv - Lq + i + 1;
+    const int n = row_keys(kv_len, b, Lq, Lkv, i);
     const unsigned int *gu =
         reinterpret_cast<const unsigned int *>(scores + (((size_t)b * Hkv + g) * row_count + r) * ld);
     int32_t *o = idx + (((size_t)b * Hkv + g) * Lq + i) * (size_t)topk;
@@ -354,7 +363,7 @@ template <bool AL>
 __global__ void __launch_bounds__(WK_WARPS * 32, 5)
 topk_warp_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv, int Hkv, int row_begin,
                  int row_count, int topk, long long n_items, int32_t *__restrict__ idx, uint32_t *__restrict__ mask,
-                 int W) {
+                 int W, const int32_t *__restrict__ kv_len) {
     __shared__ __align__(16) unsigned int hist_all[WK_WARPS][WK_BINS];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long item = (long long)blockIdx.x * WK_WARPS + warp;
@@ -363,7 +372,7 @@ topk_warp_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv
     const int r = row_count - 1 - (int)(item % row_count);
     const long long bg = item / row_count;
     const int i = row_begin + r;
-    const int n = Lkv - Lq + i + 1;
+    const int n = row_keys(kv_len, (int)(bg / Hkv), Lq, Lkv, i);
     const unsigned int *u = reinterpret_cast<const unsigned int *>(scores + ((size_t)bg * row_count + r) * ld);
     int32_t *o = idx + ((size_t)bg * Lq + i) * (size_t)topk;
     uint32_t *mrow = mask ? mask + ((size_t)bg * Lq + i) * (size_t)W : nullptr;
@@ -580,10 +589,10 @@ cudaError_t topk_launch(const Shape &s, const float *scores, long long ld, int r
         const unsigned int grid = (unsigned int)((n_items + WK_WARPS - 1) / WK_WARPS);
         if (al)
             topk_warp_kernel<true><<<grid, WK_WARPS * 32, 0, st>>>(scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin,
-                                                                   row_count, topk, n_items, idx, mask, W);
+                                                                   row_count, topk, n_items, idx, mask, W, s.kv_len);
         else
             topk_warp_kernel<false><<<grid, WK_WARPS * 32, 0, st>>>(scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin,
-                                                                    row_count, topk, n_items, idx, mask, W);
+                                                                    row_count, topk, n_items, idx, mask, W, s.kv_len);
         count_launch();
         if (mask_done) *mask_done = mask != nullptr;
         return cudaGetLastError();
@@ -596,13 +605,13 @@ cudaError_t topk_launch(const Shape &s, const float *scores, long long ld, int r
     if (split > 0) {
         const long long n_max = off + row_begin + split;
         topk_radix_kernel<true><<<dim3((unsigned)split, s.Hkv, s.B), NT, (size_t)n_max * 4, st>>>(
-            scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, 0, topk, idx); count_launch();
+            scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, 0, topk, idx, s.kv_len); count_launch();
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     if (split < row_count) {
         topk_radix_kernel<false><<<dim3((unsigned)(row_count - split), s.Hkv, s.B), NT, 0, st>>>(
-            scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, (int)split, topk, idx); count_launch();
+            scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, (int)split, topk, idx, s.kv_len); count_launch();
     }
     return cudaGetLastError();
 }

@@ -143,6 +143,27 @@ int hysparse_block(const hs_shape *shape, const void *q_full, const void *k, con
                    const float *const *gate_logit, void *const *out_sparse, int topk, int window,
                    int32_t *idx_out, int row_chunk, void *ws, size_t ws_bytes, hs_stream_t stream);
 
+/* One decode step of the hybrid block over a batch whose sequences have
+ * caches of different lengths (serving: every sequence decodes one token,
+ * each at its own position).  Same computation, arguments and layouts as
+ * hysparse_block with Lq == 1, plus
+ *   kv_len  DEVICE array of B int32, 1 <= kv_len[b] <= Lkv: sequence b's
+ *           cache is k[b, 0:kv_len[b]], v[b, 0:kv_len[b]] (the Lkv-row
+ *           buffers hold it at their start; rows past it are never read)
+ *           and its new query sits at position kv_len[b] - 1, so its full
+ *           layer, scores, top-k and window branch see exactly those keys.
+ * Requires Lq == 1 and the bf16, d = 128 path (else HS_ERR_UNSUPPORTED);
+ * kv_len must be 4-byte aligned.  The lengths live on the device, so a value
+ * outside [1, Lkv] is found there: it is clamped (nothing outside the cache
+ * is read) and HS_ERR_INVALID_ARG is recorded in the workspace status word
+ * (hysparse_workspace_status).  The whole batch is one row chunk.
+ * Errors: as hysparse_block. */
+int hysparse_block_varlen(const hs_shape *shape, const int32_t *kv_len, const void *q_full,
+                          const void *k, const void *v, void *out_full, float *lse, int n_sparse,
+                          const void *const *q_sparse, const float *const *gate_logit,
+                          void *const *out_sparse, int topk, int window, int32_t *idx_out,
+                          void *ws, size_t ws_bytes, hs_stream_t stream);
+
 /* Allocation-free variant of hysparse_full_attn_scores (the pages have no
  * counterpart; this is a deployment convenience).  Same computation,
  * arguments, layouts and errors, but no workspace: its scratch (a status

@@ -154,6 +154,28 @@ def test_block_rejects(L):
     assert f(chunk=8, wsb=ws_size(L, s, n_sparse=2, row_chunk=8) - 1) == _lib.HS_ERR_WORKSPACE
 
 
+def test_block_varlen_rejects(L):
+    """hysparse_block_varlen: decode shapes on the bf16 path only, a 4-byte
+    aligned length array, and the workspace of the fixed-length block."""
+    dec = shape(B=2, Lq=1, Lkv=300, Hq=8, Hkv=2, d=128, dtype=_lib.HS_BF16)
+    wsb = ws_size(L, dec, n_sparse=2)
+    PA = ctypes.c_void_p * 2
+    qa, ga, oa = PA(A, A + 256), PA(A + 512, A + 768), PA(A + 1024, A + 1280)
+    c = lambda x: ctypes.cast(x, ctypes.c_void_p)
+
+    def f(**kw):
+        s = kw.get("s", dec)
+        return L.hysparse_block_varlen(ctypes.byref(s), kw.get("kvl", P(8)), P(1), P(2), P(3), P(4), None, 2,
+                                       c(qa), c(ga), c(oa), kw.get("k", 8), 16, None, P(7),
+                                       kw.get("wsb", wsb), None)
+    assert f(kvl=None) == _lib.HS_ERR_INVALID_ARG
+    assert f(kvl=ctypes.c_void_p(A + 0x100000 * 8 + 2)) == _lib.HS_ERR_INVALID_ARG     # misaligned
+    assert f(s=shape(B=2, Lq=64, Lkv=300, Hq=8, Hkv=2, d=128, dtype=_lib.HS_BF16)) == _lib.HS_ERR_UNSUPPORTED
+    assert f(s=shape(B=2, Lq=1, Lkv=300, Hq=8, Hkv=2, d=64)) == _lib.HS_ERR_UNSUPPORTED   # fp32 path
+    assert f(k=0) == _lib.HS_ERR_INVALID_ARG
+    assert f(wsb=wsb - 1) == _lib.HS_ERR_WORKSPACE
+
+
 def test_workspace_status_rejects_null(L):
     assert L.hysparse_workspace_status(None, None) == _lib.HS_ERR_INVALID_ARG
 
