@@ -512,6 +512,139 @@ def bench_ours(args, w, ws_, rank, local):
     return res
 
 
+# ------------------------------------------------- decode, mixed lengths
+
+def bench_varlen(args, w, ws_, rank, local):
+    """Decode with every sequence at its own cache length (seeded, uniform in
+    [window, Lkv]) through hysparse_block_varlen.  Same timing rules as the
+    fixed-length run; the roofline is the whole block against HBM."""
+    import hybrid_sparse_attention_tcgen05_b200 as hs
+    from hybrid_sparse_attention_tcgen05_b200 import inputs as gen
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_kind = load_peaks()
+    inp = gen.make_inputs(w, seed=args.seed + rank, device=str(dev))
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    qs, gates = inp["q_sparse"], inp["gate"]
+    g = torch.Generator().manual_seed(args.seed + 1000 + rank)
+    lens = torch.randint(w.window, w.Lkv + 1, (w.B,), generator=g).to(torch.int32)
+    kv_len = lens.to(dev)
+    shape = hs.shape_of(q, k)
+    ws_full = hs.alloc_workspace(shape, w.topk, w.window, w.n_sparse, 1, dev)
+    out = torch.empty_like(q)
+    outs = [torch.empty_like(x) for x in qs]
+    lse = torch.empty(w.B, w.Hq, 1, dtype=torch.float32, device=dev)
+    idx = torch.empty(w.B, w.Hkv, 1, w.topk, dtype=torch.int32, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def block_step():
+        hs.block(q, k, v, qs, gates, w.topk, w.window, out_full=out, out_sparse=outs, idx=idx, lse=lse,
+                 ws=ws_full, kv_len=kv_len)
+
+    for _ in range(args.warmup):
+        block_step()
+    torch.cuda.synchronize()
+    st = hs.workspace_status(ws_full)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    if ws_ > 1:
+        torch.distributed.barrier()
+    step_ms = []
+    launches0 = hs.launch_count()
+    with ClockSampler(local) as clk:
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            flush.fill_(1.0)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            block_step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            step_ms.append(e0.elapsed_time(e1))
+        wall = time.perf_counter() - t0
+    gpu_launches = hs.launch_count() - launches0
+    if ws_ > 1:
+        torch.distributed.barrier()
+    ms_per_step = max_over_ranks(sum(step_ms), ws_, dev) / args.steps
+    value = w.B * ws_ / (ms_per_step / 1e3)
+
+    # end to end: each step brings the new token's queries, gates and K/V row
+    # from pinned host memory, writes the K/V row into each sequence's cache
+    # at its own position, runs the block and reads every output back
+    pin = lambda x: x.to("cpu").pin_memory()
+    rows = torch.arange(w.B, device=dev)
+    pos = kv_len.long() - 1
+    h_in = [pin(x) for x in [q, k[rows, pos].unsqueeze(1), v[rows, pos].unsqueeze(1), *qs, *gates]]
+    d_in = [torch.empty_like(x, device=dev) for x in h_in]
+    h_res = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(1 + len(qs))]
+    h2d = sum(x.numel() * x.element_size() for x in h_in)
+    d2h = sum(x.numel() * x.element_size() for x in h_res)
+    n_in = 3 + len(qs)
+
+    def e2e_step():
+        for a_, b_ in zip(d_in, h_in):
+            a_.copy_(b_, non_blocking=True)
+        k[rows, pos] = d_in[1][:, 0]
+        v[rows, pos] = d_in[2][:, 0]
+        hs.block(d_in[0], k, v, d_in[3:n_in], d_in[n_in:], w.topk, w.window, out_full=out, out_sparse=outs,
+                 idx=idx, lse=lse, ws=ws_full, kv_len=kv_len)
+        for a_, b_ in zip(h_res, [out, *outs]):
+            a_.copy_(b_, non_blocking=True)
+
+    e2e_steps = int(max(4, min(32, 1500.0 / max(ms_per_step, 1e-3))))
+    e2e_step()
+    torch.cuda.synchronize()
+    if ws_ > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, ws_, dev)
+
+    # algorithmic HBM bytes of the block: every sequence's K and V read once by
+    # the full layer, then each sparse layer's gathered rows
+    L = lens.double()
+    esz = 2
+    kv_bytes = float((2 * L * w.Hkv * w.d * esz).sum())
+    gather = float(((torch.clamp(L, max=w.topk) + torch.clamp(L, max=w.window)) * w.Hkv * 2 * w.d * esz).sum())
+    bytes_total = kv_bytes + w.n_sparse * gather
+    achieved = bytes_total / (ms_per_step / 1e3) / 1e9
+    roof = {"kernel": "hysparse_block_varlen (decode_full_mma + decode_combine + topk + n x sparse_attn_mma)",
+            "bound": "hbm", "unit": "GB/s",
+            "work": "each sequence's K and V read once (2*L_b*Hkv*d*2 B) + per sparse layer its gathered "
+                    "(min(k, L_b) + min(w, L_b)) K and V rows",
+            "achieved": achieved, "peak": peaks["hbm_gbs"], "peak_kind": f"{peak_kind} (burst)",
+            "frac": achieved / peaks["hbm_gbs"], "launch_ms": ms_per_step, "traffic": None}
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded, generated on device)",
+        "config": {"workload": f"{w.name}-varlen", "B": w.B, "Lq": 1, "Lkv_max": w.Lkv, "Hq": w.Hq,
+                   "Hkv": w.Hkv, "d": w.d, "topk": w.topk, "window": w.window, "n_sparse": w.n_sparse,
+                   "kv_len": {"min": int(lens.min()), "mean": float(L.mean()), "max": int(lens.max()),
+                              "draw": f"uniform in [{w.window}, {w.Lkv}], seed {args.seed + 1000 + rank}"},
+                   "l2": "flushed: 252 MiB written between timed steps", "parallelism": f"replicas x{ws_}"},
+        "clocks": clk.summary(),
+        "e2e": {"value": w.B * ws_ / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "api": "hybrid_sparse_attention_tcgen05_b200.block(kv_len=...); pinned host buffers; copy in, "
+                       "K/V row into each cache at its position, block, copy out, one stream",
+                "steps": e2e_steps},
+        "gpu_launches": gpu_launches,
+        "roofline": roof,
+        "decode_step_us": ms_per_step * 1e3,
+        "wall_s_timed": wall,
+    }
+
+
 # --------------------------------------------------------- CPU (oracle) arm
 
 def row_cost(w, i):
@@ -622,6 +755,8 @@ def main():
     ap.add_argument("--row-chunk", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    ap.add_argument("--varlen", action="store_true",
+                    help="decode workloads: every sequence at its own cache length (hysparse_block_varlen)")
     ap.add_argument("--seq", type=int, default=0,
                     help="override the cache length (and the prefill length) for small profiling runs")
     args = ap.parse_args()
@@ -644,6 +779,13 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=torch.device("cuda", local))
     try:
+        if args.varlen:
+            if w.Lq != 1:
+                raise SystemExit("--varlen applies to decode workloads (Lq = 1)")
+            res = bench_varlen(args, w, world, rank, local)
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return 0
         res = bench_ours(args, w, world, rank, local)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             host = oracle_inputs(w, args.seed, res.pop("_inputs"))
