@@ -28,7 +28,8 @@ from . import _lib
 from ._lib import HysparseError, HsShape
 
 __all__ = ["shape_of", "workspace_size", "alloc_workspace", "full_attn_scores", "topk",
-           "sparse_attn", "block", "workspace_status", "version", "launch_count", "HysparseError", "HsShape"]
+           "sparse_attn", "block", "block_paged", "workspace_status", "version", "launch_count",
+           "HysparseError", "HsShape"]
 
 
 def _dtype_code(t: torch.dtype) -> int:
@@ -205,6 +206,58 @@ def block(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_sparse: Sequence[
         ctypes.cast(oa, ctypes.c_void_p), int(k_top), int(window), _ptr(idx), int(row_chunk),
         _ptr(ws), ws.numel(), _stream(dev))
     _lib.check(st, "hysparse_block")
+    return out_full, lse, idx, out_sparse
+
+
+def block_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, q_sparse: Sequence[torch.Tensor],
+                gate_logit: Sequence[torch.Tensor], k_top: int, window: int, kv_len: torch.Tensor,
+                block_table: torch.Tensor, *, max_len: Optional[int] = None,
+                out_full: Optional[torch.Tensor] = None, out_sparse: Optional[List[torch.Tensor]] = None,
+                idx: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                ws: Optional[torch.Tensor] = None, scale: Optional[float] = None):
+    """One decode step over paged caches (hysparse_block_paged).
+
+    q [B,1,Hq,d]; k_pages, v_pages [num_pages,page_size,Hkv,d]; kv_len int32
+    [B]; block_table int32 [B,max_pages] (sequence b's key j is row
+    j % page_size of page block_table[b, j // page_size]).  max_len: the
+    longest cache a sequence may have (default max_pages * page_size).
+    Returns (out_full, lse, idx, [out_sparse_n])."""
+    dev = _need_cuda(q, k_pages, v_pages, kv_len, block_table, out_full, idx, lse, ws, *q_sparse, *gate_logit,
+                     *(out_sparse or []))
+    if k_pages.dim() != 4 or v_pages.shape != k_pages.shape or block_table.dim() != 2:
+        raise ValueError("k_pages, v_pages: [num_pages, page_size, Hkv, d]; block_table: [B, max_pages]")
+    if kv_len.dtype != torch.int32 or block_table.dtype != torch.int32:
+        raise TypeError("kv_len and block_table must be int32")
+    num_pages, page_size, Hkv, d = k_pages.shape
+    B, Lq, Hq, dq = q.shape
+    if Lq != 1 or dq != d or kv_len.shape != (B,) or block_table.shape[0] != B:
+        raise ValueError("q [B,1,Hq,d], kv_len [B] and block_table [B, max_pages] must agree")
+    max_pages = block_table.shape[1]
+    Lkv = max_pages * page_size if max_len is None else int(max_len)
+    s = HsShape(B, 1, Lkv, Hq, Hkv, d, _dtype_code(q.dtype), float(scale or 0.0))
+    n = len(q_sparse)
+    if len(gate_logit) != n:
+        raise ValueError("one gate tensor per sparse layer")
+    if out_full is None:
+        out_full = torch.empty_like(q)
+    if out_sparse is None:
+        out_sparse = [torch.empty_like(x) for x in q_sparse]
+    if idx is None:
+        idx = torch.empty(B, Hkv, 1, k_top, dtype=torch.int32, device=dev)
+    if lse is None:
+        lse = torch.empty(B, Hq, 1, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = alloc_workspace(s, k_top, window, n, 0, dev)
+    PA = ctypes.c_void_p * max(n, 1)
+    qa = PA(*[x.data_ptr() for x in q_sparse])
+    ga = PA(*[x.data_ptr() for x in gate_logit])
+    oa = PA(*[x.data_ptr() for x in out_sparse])
+    st = _lib.lib().hysparse_block_paged(
+        ctypes.byref(s), _ptr(kv_len), _ptr(block_table), int(page_size), int(max_pages), int(num_pages),
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(out_full), _ptr(lse), n,
+        ctypes.cast(qa, ctypes.c_void_p), ctypes.cast(ga, ctypes.c_void_p), ctypes.cast(oa, ctypes.c_void_p),
+        int(k_top), int(window), _ptr(idx), _ptr(ws), ws.numel(), _stream(dev))
+    _lib.check(st, "hysparse_block_paged")
     return out_full, lse, idx, out_sparse
 
 

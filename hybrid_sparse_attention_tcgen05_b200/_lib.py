@@ -30,6 +30,7 @@ EXPORTS = (
     "hysparse_sparse_attn",
     "hysparse_block",
     "hysparse_block_varlen",
+    "hysparse_block_paged",
     "hysparse_full_attn_scores_noalloc",
     "hysparse_workspace_status",
     "hysparse_selftest_exp2",
@@ -78,6 +79,8 @@ def lib():
     L.hysparse_block.restype = I
     L.hysparse_block_varlen.argtypes = [SP, P, P, P, P, P, P, I, P, P, P, I, I, P, P, SZ, P]
     L.hysparse_block_varlen.restype = I
+    L.hysparse_block_paged.argtypes = [SP, P, P, I, I, I, P, P, P, P, P, I, P, P, P, I, I, P, P, SZ, P]
+    L.hysparse_block_paged.restype = I
     L.hysparse_full_attn_scores_noalloc.argtypes = [SP, P, P, P, P, P, P, LL, I, I, P]
     L.hysparse_full_attn_scores_noalloc.restype = I
     L.hysparse_selftest_exp2.argtypes = [P, P, P, I, P]

@@ -247,9 +247,16 @@ int hysparse_sparse_attn(const hs_shape *shape, const void *q, const void *k, co
 }
 
 namespace {
-// hysparse_block, and hysparse_block_varlen when kv_len is set
-int block_impl(const hs_shape *shape, const int32_t *kv_len, const void *q_full, const void *k, const void *v,
-               void *out_full, float *lse, int n_sparse, const void *const *q_sparse,
+// Paged caches: where the pages are and how sequences map onto them.
+struct Paging {
+    const int32_t *table = nullptr;
+    int page_size = 0, max_pages = 0, num_pages = 0;
+};
+
+// hysparse_block; hysparse_block_varlen when kv_len is set; and
+// hysparse_block_paged when the paging table is set too
+int block_impl(const hs_shape *shape, const int32_t *kv_len, const Paging &pg, const void *q_full, const void *k,
+               const void *v, void *out_full, float *lse, int n_sparse, const void *const *q_sparse,
                const float *const *gate_logit, void *const *out_sparse, int topk, int window,
                int32_t *idx_out, int row_chunk, void *ws, size_t ws_bytes, hs_stream_t stream) {
     Shape s;
@@ -260,6 +267,19 @@ int block_impl(const hs_shape *shape, const int32_t *kv_len, const void *q_full,
         if (s.Lq != 1 || !use_decode_path(s)) return HS_ERR_UNSUPPORTED;
         if ((reinterpret_cast<uintptr_t>(kv_len) & 3u) != 0) return HS_ERR_INVALID_ARG;
         s.kv_len = kv_len;
+    }
+    if (pg.table != nullptr) {
+        if (kv_len == nullptr) return HS_ERR_INVALID_ARG;
+        const int ps = pg.page_size;
+        if (ps < 1 || ps > (1 << 16) || (ps & (ps - 1)) != 0) return HS_ERR_INVALID_ARG;
+        if (pg.max_pages < 1 || pg.num_pages < 1) return HS_ERR_INVALID_ARG;
+        if ((long long)pg.max_pages * ps < s.Lkv) return HS_ERR_INVALID_ARG;           // table too short
+        if ((long long)pg.num_pages * ps > 0x7fffffffLL) return HS_ERR_INVALID_ARG;    // pool rows in int32
+        if ((reinterpret_cast<uintptr_t>(pg.table) & 3u) != 0) return HS_ERR_INVALID_ARG;
+        s.block_table = pg.table;
+        s.page_shift = __builtin_ctz((unsigned)ps);
+        s.max_pages = pg.max_pages;
+        s.num_pages = pg.num_pages;
     }
     if (topk < 1 || topk > kMaxTopk || window < 1 || window > kMaxWindow || n_sparse < 0)
         return HS_ERR_INVALID_ARG;
@@ -315,8 +335,8 @@ int hysparse_block(const hs_shape *shape, const void *q_full, const void *k, con
                    const float *const *gate_logit, void *const *out_sparse, int topk, int window,
                    int32_t *idx_out, int row_chunk, void *ws, size_t ws_bytes,
                    hs_stream_t stream) {
-    return block_impl(shape, nullptr, q_full, k, v, out_full, lse, n_sparse, q_sparse, gate_logit, out_sparse,
-                      topk, window, idx_out, row_chunk, ws, ws_bytes, stream);
+    return block_impl(shape, nullptr, Paging{}, q_full, k, v, out_full, lse, n_sparse, q_sparse, gate_logit,
+                      out_sparse, topk, window, idx_out, row_chunk, ws, ws_bytes, stream);
 }
 
 int hysparse_block_varlen(const hs_shape *shape, const int32_t *kv_len, const void *q_full, const void *k,
@@ -324,8 +344,23 @@ int hysparse_block_varlen(const hs_shape *shape, const int32_t *kv_len, const vo
                           const float *const *gate_logit, void *const *out_sparse, int topk, int window,
                           int32_t *idx_out, void *ws, size_t ws_bytes, hs_stream_t stream) {
     if (kv_len == nullptr) return HS_ERR_INVALID_ARG;
-    return block_impl(shape, kv_len, q_full, k, v, out_full, lse, n_sparse, q_sparse, gate_logit, out_sparse,
-                      topk, window, idx_out, 0, ws, ws_bytes, stream);
+    return block_impl(shape, kv_len, Paging{}, q_full, k, v, out_full, lse, n_sparse, q_sparse, gate_logit,
+                      out_sparse, topk, window, idx_out, 0, ws, ws_bytes, stream);
+}
+
+int hysparse_block_paged(const hs_shape *shape, const int32_t *kv_len, const int32_t *block_table, int page_size,
+                         int max_pages, int num_pages, const void *q_full, const void *k_pages,
+                         const void *v_pages, void *out_full, float *lse, int n_sparse,
+                         const void *const *q_sparse, const float *const *gate_logit, void *const *out_sparse,
+                         int topk, int window, int32_t *idx_out, void *ws, size_t ws_bytes, hs_stream_t stream) {
+    if (kv_len == nullptr || block_table == nullptr) return HS_ERR_INVALID_ARG;
+    Paging pg;
+    pg.table = block_table;
+    pg.page_size = page_size;
+    pg.max_pages = max_pages;
+    pg.num_pages = num_pages;
+    return block_impl(shape, kv_len, pg, q_full, k_pages, v_pages, out_full, lse, n_sparse, q_sparse, gate_logit,
+                      out_sparse, topk, window, idx_out, 0, ws, ws_bytes, stream);
 }
 
 int hysparse_workspace_status(void *ws, hs_stream_t stream) {

@@ -22,6 +22,12 @@ struct Shape {
     // sequence b's cache length (its new token at position kv_len[b] - 1);
     // NULL = every sequence has Lkv.  Only the bf16 decode path reads it.
     const int32_t *kv_len = nullptr;
+    // paged caches (decode): k and v are pools of num_pages pages of
+    // 2^page_shift rows [page][row][Hkv][d]; key j of sequence b lives in page
+    // block_table[b * max_pages + (j >> page_shift)] (device, int32).  NULL:
+    // contiguous [B][Lkv][Hkv][d] caches.
+    const int32_t *block_table = nullptr;
+    int page_shift = 0, max_pages = 0, num_pages = 0;
     int G() const { return Hq / Hkv; }
 };
 

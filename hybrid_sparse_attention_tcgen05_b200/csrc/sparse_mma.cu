@@ -74,6 +74,11 @@ struct SpParams {
     unsigned int *status;
     unsigned long long wait_ns;
     const int32_t *kv_len;   // [B] cache lengths (decode over caches of different lengths) or NULL
+    // paged caches (decode): k and v are pools of num_pages pages of 2^page_shift
+    // rows; key j of sequence b is row j & (2^page_shift - 1) of page
+    // block_table[b * max_pages + (j >> page_shift)].  NULL: contiguous caches.
+    const int32_t *block_table;
+    int page_shift, max_pages, num_pages;
 };
 
 // Cache length of sequence b: kv_len[b] when given (a value outside
@@ -101,7 +106,8 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // then copied two per instruction (16 lanes x 16 bytes per 256-byte row).
 __device__ __forceinline__ void issue_chunk(const SpParams &p, const int32_t *list, bool from_list, int lo,
                                             int n_list, int t0, int pos, const __nv_bfloat16 *kb,
-                                            const __nv_bfloat16 *vb, uint8_t *stage, uint32_t &vmask, int lane) {
+                                            const __nv_bfloat16 *vb, uint8_t *stage, uint32_t &vmask, int lane,
+                                            const int32_t *table) {
     const int t = t0 + lane;
     int key = -1;
     if (t < n_list) {
@@ -109,6 +115,18 @@ __device__ __forceinline__ void issue_chunk(const SpParams &p, const int32_t *li
         if (key < -1 || key > pos) {
             report(p.status, HS_ERR_INVALID_INDEX);
             key = -1;
+        }
+    }
+    // row of the key in the cache (kb, vb): the key itself, or its row in the
+    // page pool when the cache is paged (a page outside the pool is reported
+    // and the key dropped, like an invalid index)
+    if (table != nullptr && key >= 0) {
+        const int page = __ldg(table + (key >> p.page_shift));
+        if (page < 0 || page >= p.num_pages) {
+            report(p.status, HS_ERR_INVALID_INDEX);
+            key = -1;
+        } else {
+            key = (page << p.page_shift) | (key & ((1 << p.page_shift) - 1));
         }
     }
     vmask = __ballot_sync(0xffffffffu, key >= 0);
@@ -130,7 +148,7 @@ __device__ __forceinline__ void issue_chunk(const SpParams &p, const int32_t *li
 template <int NB>
 __device__ __forceinline__ void compute_chunk(const uint8_t *stage, uint32_t vmask, const uint32_t (&bq)[NB][8][2],
                                               float c2, Branch<NB> &br, int lane, float *stash = nullptr,
-                                              long long stash_ld = 0, int j0 = 0, int G = 0) {
+                                              long long stash_ld = 0, int j0 = 0, int G = 0, int j_lim = 0) {
     const uint32_t ks_base = smem_u32(stage);
     const uint32_t vs_base = smem_u32(stage + CH * RS);
     float c[NB][2][4];
@@ -173,9 +191,12 @@ __device__ __forceinline__ void compute_chunk(const uint8_t *stage, uint32_t vma
                     x[mt][rh] = kv[mt][rh] ? c[nb][mt][2 * rh + e] * c2 : -INFINITY;
                     cm = fmaxf(cm, x[mt][rh]);
                     if (stash != nullptr) {
+                        // every key of the range, -inf for one that was dropped (a page
+                        // outside the pool), so that its score is 0 and no stale value
+                        // is read back; rows past the range are not written
                         const int h = 8 * nb + 2 * (lane & 3) + e;
-                        if (h < G && kv[mt][rh])
-                            stash[(long long)h * stash_ld + j0 + 16 * mt + (lane >> 2) + 8 * rh] = x[mt][rh];
+                        const int rr = 16 * mt + (lane >> 2) + 8 * rh;
+                        if (h < G && rr < j_lim) stash[(long long)h * stash_ld + j0 + rr] = x[mt][rh];
                     }
                 }
             cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 4));
@@ -230,6 +251,7 @@ struct WarpCtx {
     const SpParams *p;
     const int32_t *list;
     const __nv_bfloat16 *kb, *vb;
+    const int32_t *table = nullptr;   // this sequence's block table row (paged caches) or NULL
     uint8_t *wbase;
     int lo, pos, lane;
     float c2;
@@ -260,7 +282,7 @@ __device__ __forceinline__ void run_branch(const WarpCtx &w, bool from_list, con
         uint32_t vmask = 0;
         if (c < nch) {
             issue_chunk(p, w.list, from_list, w.lo, n_list, c * CH, w.pos, w.kb, w.vb, w.wbase + s * STAGE_BYTES,
-                        vmask, w.lane);
+                        vmask, w.lane, w.table);
         } else {
             cp_async_commit();
         }
@@ -275,7 +297,7 @@ __device__ __forceinline__ void run_branch(const WarpCtx &w, bool from_list, con
         __syncwarp();
         const int s = c % ST;
         compute_chunk<NB>(w.wbase + s * STAGE_BYTES, pick3(s, vm0, vm1, vm2), bq, w.c2, br, w.lane, w.stash,
-                          w.stash_ld, w.lo + c * CH, w.G);
+                          w.stash_ld, w.lo + c * CH, w.G, n_list - c * CH);
     }
     cp_async_wait<0>();
     __syncwarp();
@@ -316,8 +338,14 @@ __global__ void __launch_bounds__(SW * 32, 1) sparse_attn_mma(const SpParams p) 
 
     WarpCtx w;
     w.p = &p;
-    w.kb = p.k + ((size_t)b * p.Lkv * p.Hkv + g) * 128;
-    w.vb = p.v + ((size_t)b * p.Lkv * p.Hkv + g) * 128;
+    if (p.block_table != nullptr) {   // paged: rows of the page pool, located through the table
+        w.kb = p.k + (size_t)g * 128;
+        w.vb = p.v + (size_t)g * 128;
+        w.table = p.block_table + (size_t)b * p.max_pages;
+    } else {
+        w.kb = p.k + ((size_t)b * p.Lkv * p.Hkv + g) * 128;
+        w.vb = p.v + ((size_t)b * p.Lkv * p.Hkv + g) * 128;
+    }
     w.list = p.idx + (((size_t)b * p.Hkv + g) * p.Lq + i) * p.topk;
     w.wbase = wbase;
     w.lo = max(0, pos - p.window + 1);
@@ -424,8 +452,14 @@ __global__ void __launch_bounds__(SW * 32, 1) decode_full_mma(const DecParams dp
     const int hi = min(Lb, lo + kDecChunk);
     WarpCtx w;
     w.p = &p;
-    w.kb = p.k + ((size_t)b * p.Lkv * p.Hkv + g) * 128;
-    w.vb = p.v + ((size_t)b * p.Lkv * p.Hkv + g) * 128;
+    if (p.block_table != nullptr) {   // paged: rows of the page pool, located through the table
+        w.kb = p.k + (size_t)g * 128;
+        w.vb = p.v + (size_t)g * 128;
+        w.table = p.block_table + (size_t)b * p.max_pages;
+    } else {
+        w.kb = p.k + ((size_t)b * p.Lkv * p.Hkv + g) * 128;
+        w.vb = p.v + ((size_t)b * p.Lkv * p.Hkv + g) * 128;
+    }
     w.list = nullptr;
     w.wbase = wbase;
     w.lo = lo;
@@ -541,7 +575,8 @@ cudaError_t sparse_attn_mma_launch(const Shape &s, const void *q, const void *k,
                                    cudaStream_t st) {
     tc::SpParams p{(const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, idx, gate,
                    (__nv_bfloat16 *)out, (__nv_bfloat16 *)og, (__nv_bfloat16 *)ol, s.B, s.Lq, s.Lkv, s.Hq,
-                   s.Hkv, s.G(), topk, window, s.scale * kLog2e, status, wait_ns, s.kv_len};
+                   s.Hkv, s.G(), topk, window, s.scale * kLog2e, status, wait_ns, s.kv_len,
+                   s.block_table, s.page_shift, s.max_pages, s.num_pages};
     return s.G() <= 8 ? tc::launch_nb<1>(p, st) : tc::launch_nb<2>(p, st);
 }
 
@@ -561,7 +596,8 @@ cudaError_t decode_full_mma_launch(const Shape &s, const void *q, const void *k,
     tc::DecParams dp;
     dp.sp = tc::SpParams{(const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, nullptr,
                          nullptr, (__nv_bfloat16 *)out, nullptr, nullptr, s.B, 1, s.Lkv, s.Hq, s.Hkv, s.G(),
-                         1, 1, s.scale * kLog2e, status, 0, s.kv_len};
+                         1, 1, s.scale * kLog2e, status, 0, s.kv_len,
+                         s.block_table, s.page_shift, s.max_pages, s.num_pages};
     dp.part_o = reinterpret_cast<float *>(w);
     w += align_up(rows * nchunk * 128 * sizeof(float), 256);
     dp.part_ml = reinterpret_cast<float2 *>(w);

@@ -164,6 +164,26 @@ int hysparse_block_varlen(const hs_shape *shape, const int32_t *kv_len, const vo
                           void *const *out_sparse, int topk, int window, int32_t *idx_out,
                           void *ws, size_t ws_bytes, hs_stream_t stream);
 
+/* hysparse_block_varlen over paged caches: k_pages and v_pages are pools of
+ * num_pages pages, each page_size rows of [Hkv][d] ([num_pages][page_size]
+ * [Hkv][d], bf16), and sequence b's key j is row j % page_size of page
+ * block_table[b * max_pages + j / page_size] (block_table: DEVICE int32,
+ * B rows of max_pages entries, 4-byte aligned).  Only the entries that cover
+ * keys 0 .. kv_len[b]-1 are read.  page_size is a power of two in
+ * [1, 65536]; max_pages * page_size >= Lkv (shape->Lkv is the longest cache
+ * any sequence may have) and num_pages * page_size < 2^31.  A table entry
+ * outside [0, num_pages) is found on the device: the key is dropped and
+ * HS_ERR_INVALID_INDEX recorded in the workspace status word.  The
+ * workspace is the one hysparse_workspace_size gives for the shape.
+ * Errors: as hysparse_block_varlen, HS_ERR_INVALID_ARG for the paging
+ * arguments. */
+int hysparse_block_paged(const hs_shape *shape, const int32_t *kv_len, const int32_t *block_table,
+                         int page_size, int max_pages, int num_pages, const void *q_full,
+                         const void *k_pages, const void *v_pages, void *out_full, float *lse,
+                         int n_sparse, const void *const *q_sparse, const float *const *gate_logit,
+                         void *const *out_sparse, int topk, int window, int32_t *idx_out, void *ws,
+                         size_t ws_bytes, hs_stream_t stream);
+
 /* Allocation-free variant of hysparse_full_attn_scores (the pages have no
  * counterpart; this is a deployment convenience).  Same computation,
  * arguments, layouts and errors, but no workspace: its scratch (a status

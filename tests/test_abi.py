@@ -176,6 +176,31 @@ def test_block_varlen_rejects(L):
     assert f(wsb=wsb - 1) == _lib.HS_ERR_WORKSPACE
 
 
+def test_block_paged_rejects(L):
+    """hysparse_block_paged: a power-of-two page size, a table long enough for
+    Lkv, a pool whose rows fit in int32, aligned lengths and table."""
+    dec = shape(B=2, Lq=1, Lkv=300, Hq=8, Hkv=2, d=128, dtype=_lib.HS_BF16)
+    wsb = ws_size(L, dec, n_sparse=2)
+    PA = ctypes.c_void_p * 2
+    qa, ga, oa = PA(A, A + 256), PA(A + 512, A + 768), PA(A + 1024, A + 1280)
+    c = lambda x: ctypes.cast(x, ctypes.c_void_p)
+
+    def f(**kw):
+        s = kw.get("s", dec)
+        return L.hysparse_block_paged(ctypes.byref(s), kw.get("kvl", P(8)), kw.get("tab", P(9)),
+                                      kw.get("ps", 64), kw.get("mp", 5), kw.get("np", 100), P(1), P(2), P(3),
+                                      P(4), None, 2, c(qa), c(ga), c(oa), 8, 16, None, P(7), wsb, None)
+    assert f(tab=None) == _lib.HS_ERR_INVALID_ARG
+    assert f(kvl=None) == _lib.HS_ERR_INVALID_ARG
+    assert f(ps=48) == _lib.HS_ERR_INVALID_ARG                       # not a power of two
+    assert f(ps=0) == _lib.HS_ERR_INVALID_ARG
+    assert f(mp=4) == _lib.HS_ERR_INVALID_ARG                        # 4 * 64 < Lkv = 300
+    assert f(np=0) == _lib.HS_ERR_INVALID_ARG
+    assert f(ps=1 << 16, np=1 << 16) == _lib.HS_ERR_INVALID_ARG      # pool rows past int32
+    assert f(tab=ctypes.c_void_p(A + 0x100000 * 9 + 2)) == _lib.HS_ERR_INVALID_ARG
+    assert f(s=shape(B=2, Lq=64, Lkv=300, Hq=8, Hkv=2, d=128, dtype=_lib.HS_BF16)) == _lib.HS_ERR_UNSUPPORTED
+
+
 def test_workspace_status_rejects_null(L):
     assert L.hysparse_workspace_status(None, None) == _lib.HS_ERR_INVALID_ARG
 

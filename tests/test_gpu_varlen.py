@@ -1,7 +1,9 @@
-"""Decode over caches of different lengths (hysparse_block_varlen) on the
-GPU: every sequence must get exactly what a fixed-length decode over its own
-cache gives, and match the oracle; lengths outside [1, Lkv] are reported
-through the workspace status word without any read outside the cache."""
+"""Decode over caches of different lengths (hysparse_block_varlen) and over
+paged caches (hysparse_block_paged) on the GPU: every sequence must get
+exactly what a fixed-length decode over its own contiguous cache gives, and
+match the oracle; lengths outside [1, Lkv] and pages outside the pool are
+reported through the workspace status word without any read outside the
+cache."""
 import pytest
 import torch
 
@@ -84,3 +86,61 @@ def test_varlen_lengths_outside_the_cache_are_reported():
     good = torch.tensor(LENS, dtype=torch.int32, device=DEV)
     hs.block(inp["q"], inp["k"], inp["v"], inp["q_sparse"], inp["gate"], TOPK, WINDOW, ws=ws, kv_len=good)
     assert hs.workspace_status(ws) == _lib.HS_OK
+
+
+def _paged(k, v, lens, page_size, seed=9, spare=7):
+    """Scatter the contiguous caches into shuffled pages: pools
+    [num_pages, page_size, Hkv, d] and the block table [B, max_pages]."""
+    B, Lkv, Hkv, d = k.shape
+    max_pages = (Lkv + page_size - 1) // page_size
+    need = [(L + page_size - 1) // page_size for L in lens]
+    num_pages = sum(need) + spare
+    g = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(num_pages, generator=g).tolist()
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    kp = torch.zeros(num_pages, page_size, Hkv, d, dtype=k.dtype, device=k.device)
+    vp = torch.zeros_like(kp)
+    nxt = 0
+    for b, L in enumerate(lens):
+        for pg in range(need[b]):
+            page = perm[nxt]
+            nxt += 1
+            table[b, pg] = page
+            lo, hi = pg * page_size, min(L, (pg + 1) * page_size)
+            kp[page, : hi - lo] = k[b, lo:hi]
+            vp[page, : hi - lo] = v[b, lo:hi]
+    return kp, vp, table.to(k.device)
+
+
+@pytest.mark.parametrize("page_size", [16, 64, 256])
+def test_paged_decode_equals_contiguous(page_size):
+    w, inp = _inputs(seed=8)
+    kv_len = torch.tensor(LENS, dtype=torch.int32, device=DEV)
+    out, lse, idx, outs = hs.block(inp["q"], inp["k"], inp["v"], inp["q_sparse"], inp["gate"], TOPK, WINDOW,
+                                   kv_len=kv_len)
+    kp, vp, table = _paged(inp["k"], inp["v"], LENS, page_size)
+    shape = hs.HsShape(w.B, 1, LKV, w.Hq, w.Hkv, w.d, 1, 0.0)
+    ws = hs.alloc_workspace(shape, TOPK, WINDOW, 2, 0, DEV)
+    po, pl, pi, ps = hs.block_paged(inp["q"], kp, vp, inp["q_sparse"], inp["gate"], TOPK, WINDOW, kv_len, table,
+                                    max_len=LKV, ws=ws)
+    assert hs.workspace_status(ws) == _lib.HS_OK
+    assert torch.equal(po, out)
+    assert torch.equal(pl, lse)
+    assert torch.equal(pi, idx)
+    for n in range(w.n_sparse):
+        assert torch.equal(ps[n], outs[n])
+
+
+def test_paged_page_outside_the_pool_is_reported():
+    w, inp = _inputs(seed=9)
+    kv_len = torch.tensor(LENS, dtype=torch.int32, device=DEV)
+    kp, vp, table = _paged(inp["k"], inp["v"], LENS, 64)
+    table[-1, 3] = kp.shape[0]            # a page covering valid keys of the last sequence
+    shape = hs.HsShape(w.B, 1, LKV, w.Hq, w.Hkv, w.d, 1, 0.0)
+    ws = hs.alloc_workspace(shape, TOPK, WINDOW, 2, 0, DEV)
+    po, _, _, ps = hs.block_paged(inp["q"], kp, vp, inp["q_sparse"], inp["gate"], TOPK, WINDOW, kv_len, table,
+                                  max_len=LKV, ws=ws)
+    assert hs.workspace_status(ws) == _lib.HS_ERR_INVALID_INDEX
+    assert torch.isfinite(po.float()).all()
+    for x in ps:
+        assert torch.isfinite(x.float()).all()
