@@ -539,9 +539,38 @@ def bench_varlen(args, w, ws_, rank, local):
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    P = args.page_size
+    if P > 0:
+        # paged caches: every sequence's pages scattered over a shuffled pool
+        if P & (P - 1):
+            raise SystemExit("--page-size must be a power of two")
+        max_pages = (w.Lkv + P - 1) // P
+        need = [(int(x) + P - 1) // P for x in lens]
+        perm = torch.randperm(sum(need), generator=g).tolist()
+        table_h = torch.full((w.B, max_pages), -1, dtype=torch.int32)
+        kp = torch.zeros(sum(need), P, w.Hkv, w.d, dtype=k.dtype, device=dev)
+        vp = torch.zeros_like(kp)
+        nxt = 0
+        for b_ in range(w.B):
+            for pg in range(need[b_]):
+                page = perm[nxt]
+                nxt += 1
+                table_h[b_, pg] = page
+                lo_, hi_ = pg * P, min(int(lens[b_]), (pg + 1) * P)
+                kp[page, : hi_ - lo_] = k[b_, lo_:hi_]
+                vp[page, : hi_ - lo_] = v[b_, lo_:hi_]
+        table = table_h.to(dev)
+
+    def run_block(qq, qq_s, gg):
+        if P > 0:
+            hs.block_paged(qq, kp, vp, qq_s, gg, w.topk, w.window, kv_len, table, max_len=w.Lkv, out_full=out,
+                           out_sparse=outs, idx=idx, lse=lse, ws=ws_full)
+        else:
+            hs.block(qq, k, v, qq_s, gg, w.topk, w.window, out_full=out, out_sparse=outs, idx=idx, lse=lse,
+                     ws=ws_full, kv_len=kv_len)
+
     def block_step():
-        hs.block(q, k, v, qs, gates, w.topk, w.window, out_full=out, out_sparse=outs, idx=idx, lse=lse,
-                 ws=ws_full, kv_len=kv_len)
+        run_block(q, qs, gates)
 
     for _ in range(args.warmup):
         block_step()
@@ -584,13 +613,20 @@ def bench_varlen(args, w, ws_, rank, local):
     d2h = sum(x.numel() * x.element_size() for x in h_res)
     n_in = 3 + len(qs)
 
+    if P > 0:   # where each sequence's new row lives in the page pool
+        prow = table[rows, pos // P].long()
+        pcol = pos % P
+
     def e2e_step():
         for a_, b_ in zip(d_in, h_in):
             a_.copy_(b_, non_blocking=True)
-        k[rows, pos] = d_in[1][:, 0]
-        v[rows, pos] = d_in[2][:, 0]
-        hs.block(d_in[0], k, v, d_in[3:n_in], d_in[n_in:], w.topk, w.window, out_full=out, out_sparse=outs,
-                 idx=idx, lse=lse, ws=ws_full, kv_len=kv_len)
+        if P > 0:
+            kp[prow, pcol] = d_in[1][:, 0]
+            vp[prow, pcol] = d_in[2][:, 0]
+        else:
+            k[rows, pos] = d_in[1][:, 0]
+            v[rows, pos] = d_in[2][:, 0]
+        run_block(d_in[0], d_in[3:n_in], d_in[n_in:])
         for a_, b_ in zip(h_res, [out, *outs]):
             a_.copy_(b_, non_blocking=True)
 
@@ -616,7 +652,8 @@ def bench_varlen(args, w, ws_, rank, local):
     gather = float(((torch.clamp(L, max=w.topk) + torch.clamp(L, max=w.window)) * w.Hkv * 2 * w.d * esz).sum())
     bytes_total = kv_bytes + w.n_sparse * gather
     achieved = bytes_total / (ms_per_step / 1e3) / 1e9
-    roof = {"kernel": "hysparse_block_varlen (decode_full_mma + decode_combine + topk + n x sparse_attn_mma)",
+    roof = {"kernel": ("hysparse_block_paged" if P > 0 else "hysparse_block_varlen")
+                      + " (decode_full_mma + decode_combine + topk + n x sparse_attn_mma)",
             "bound": "hbm", "unit": "GB/s",
             "work": "each sequence's K and V read once (2*L_b*Hkv*d*2 B) + per sparse layer its gathered "
                     "(min(k, L_b) + min(w, L_b)) K and V rows",
@@ -627,7 +664,8 @@ def bench_varlen(args, w, ws_, rank, local):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded, generated on device)",
-        "config": {"workload": f"{w.name}-varlen", "B": w.B, "Lq": 1, "Lkv_max": w.Lkv, "Hq": w.Hq,
+        "config": {"workload": f"{w.name}-varlen" + (f"-paged{P}" if P > 0 else ""), "B": w.B, "Lq": 1,
+                   "Lkv_max": w.Lkv, "Hq": w.Hq, "page_size": P if P > 0 else None,
                    "Hkv": w.Hkv, "d": w.d, "topk": w.topk, "window": w.window, "n_sparse": w.n_sparse,
                    "kv_len": {"min": int(lens.min()), "mean": float(L.mean()), "max": int(lens.max()),
                               "draw": f"uniform in [{w.window}, {w.Lkv}], seed {args.seed + 1000 + rank}"},
@@ -757,6 +795,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--varlen", action="store_true",
                     help="decode workloads: every sequence at its own cache length (hysparse_block_varlen)")
+    ap.add_argument("--page-size", type=int, default=0,
+                    help="with --varlen: paged caches of this many rows per page (hysparse_block_paged)")
     ap.add_argument("--seq", type=int, default=0,
                     help="override the cache length (and the prefill length) for small profiling runs")
     args = ap.parse_args()
