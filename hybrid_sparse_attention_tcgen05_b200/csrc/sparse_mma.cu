@@ -28,14 +28,19 @@ namespace hs {
 namespace tc {
 namespace {
 
-constexpr int SW = 4;             // warps (items) per CTA
 constexpr int CH = 32;            // keys per chunk (one per lane)
-constexpr int ST = 3;             // pipeline stages per warp
 constexpr int RS = 272;           // padded row stride in shared memory (bytes)
 constexpr int STAGE_BYTES = 2 * CH * RS;
 
+// Per head-block count NB (heads padded to 8*NB): SW warps (items) per CTA,
+// each with an ST-stage chunk ring and its Q staging.  Groups of up to 8
+// heads keep three stages (4 warps); 16-head groups trade a stage for a
+// fifth warp on the SM (measured: 3 % faster at the 64k, 16-head workload,
+// 5 % slower for 4-head decode).
 template <int NB>
 struct SpSmem {
+    static constexpr int SW = NB == 1 ? 4 : 5;
+    static constexpr int ST = NB == 1 ? 3 : 2;
     static constexpr int QB = 8 * NB * RS;               // Q staging / output staging
     static constexpr int WARP_BYTES = ST * STAGE_BYTES + QB;
     static constexpr size_t bytes = (size_t)SW * WARP_BYTES;
@@ -271,7 +276,8 @@ __device__ __forceinline__ uint32_t pick3(int s, uint32_t a, uint32_t b, uint32_
 template <int NB>
 __device__ __forceinline__ void run_branch(const WarpCtx &w, bool from_list, const uint32_t (&bq)[NB][8][2],
                                            Branch<NB> &br) {
-    static_assert(ST == 3, "pick3 assumes three stages");
+    constexpr int ST = SpSmem<NB>::ST;
+    static_assert(ST == 2 || ST == 3, "pick3 holds two or three stages");
     const SpParams &p = *w.p;
     br.init();
     const int n_list = from_list ? p.topk : w.pos - w.lo + 1;
@@ -304,10 +310,10 @@ __device__ __forceinline__ void run_branch(const WarpCtx &w, bool from_list, con
 }
 
 template <int NB>
-__global__ void __launch_bounds__(SW * 32, 1) sparse_attn_mma(const SpParams p) {
+__global__ void __launch_bounds__(SpSmem<NB>::SW * 32, 1) sparse_attn_mma(const SpParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long item = (long long)blockIdx.x * SW + warp;
+    const long long item = (long long)blockIdx.x * SpSmem<NB>::SW + warp;
     if (item >= (long long)p.B * p.Lq * p.Hkv) return;   // whole warp leaves together
     // KV head slowest, then batch, then row: neighbouring warps gather from
     // the same KV head's cache (which stays in L2) and have similar row lengths
@@ -318,7 +324,7 @@ __global__ void __launch_bounds__(SW * 32, 1) sparse_attn_mma(const SpParams p) 
     const int G = p.G;
     const int pos = seq_len(p, b) - p.Lq + i;
     uint8_t *wbase = smem + warp * SpSmem<NB>::WARP_BYTES;
-    uint8_t *qs = wbase + ST * STAGE_BYTES;
+    uint8_t *qs = wbase + SpSmem<NB>::ST * STAGE_BYTES;
     // stage the group's query rows (zero rows pad the heads up to 8*NB)
     const size_t qrow = ((size_t)b * p.Lq + i) * p.Hq + (size_t)g * G;
     for (int e = lane; e < 8 * NB * 16; e += 32) {
@@ -419,11 +425,11 @@ struct DecParams {
 };
 
 template <int NB>
-__global__ void __launch_bounds__(SW * 32, 1) decode_full_mma(const DecParams dp) {
+__global__ void __launch_bounds__(SpSmem<NB>::SW * 32, 1) decode_full_mma(const DecParams dp) {
     extern __shared__ __align__(128) uint8_t smem[];
     const SpParams &p = dp.sp;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long item = (long long)blockIdx.x * SW + warp;
+    const long long item = (long long)blockIdx.x * SpSmem<NB>::SW + warp;
     if (item >= (long long)p.B * p.Hkv * dp.nchunk) return;
     const int ch = (int)(item % dp.nchunk);
     const long long bg = item / dp.nchunk;
@@ -431,7 +437,7 @@ __global__ void __launch_bounds__(SW * 32, 1) decode_full_mma(const DecParams dp
     const int b = (int)(bg / p.Hkv);
     const int G = p.G;
     uint8_t *wbase = smem + warp * SpSmem<NB>::WARP_BYTES;
-    uint8_t *qs = wbase + ST * STAGE_BYTES;
+    uint8_t *qs = wbase + SpSmem<NB>::ST * STAGE_BYTES;
     const size_t qrow = (size_t)b * p.Hq + (size_t)g * G;      // Lq == 1
     for (int e = lane; e < 8 * NB * 16; e += 32) {
         const int h = e >> 4, cc = e & 15;
@@ -539,9 +545,9 @@ cudaError_t launch_decode(const DecParams &dp, float *lse, float *scores, long l
         attr = true;
     }
     const long long items = (long long)dp.sp.B * dp.sp.Hkv * dp.nchunk;
-    const long long blocks = (items + SW - 1) / SW;
+    const long long blocks = (items + SpSmem<NB>::SW - 1) / SpSmem<NB>::SW;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-    decode_full_mma<NB><<<(unsigned)blocks, SW * 32, SpSmem<NB>::bytes, st>>>(dp); count_launch();
+    decode_full_mma<NB><<<(unsigned)blocks, SpSmem<NB>::SW * 32, SpSmem<NB>::bytes, st>>>(dp); count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     decode_combine<<<dim3(dp.sp.Hkv, dp.sp.B), 256, 0, st>>>(dp, lse, scores, ld); count_launch();
@@ -558,9 +564,9 @@ cudaError_t launch_nb(const SpParams &p, cudaStream_t st) {
         attr = true;
     }
     const long long items = (long long)p.B * p.Lq * p.Hkv;
-    const long long blocks = (items + SW - 1) / SW;
+    const long long blocks = (items + SpSmem<NB>::SW - 1) / SpSmem<NB>::SW;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-    sparse_attn_mma<NB><<<(unsigned)blocks, SW * 32, SpSmem<NB>::bytes, st>>>(p); count_launch();
+    sparse_attn_mma<NB><<<(unsigned)blocks, SpSmem<NB>::SW * 32, SpSmem<NB>::bytes, st>>>(p); count_launch();
     return cudaGetLastError();
 }
 
