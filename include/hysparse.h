@@ -15,7 +15,8 @@
  *   B batch, Lq query rows, Lkv cache length, Hq query heads, Hkv KV heads,
  *   d head dim, G = Hq / Hkv (query head h reads KV head h / G),
  *   pos(i) = Lkv - Lq + i  (causal, bottom-right aligned: row i sees keys
- *   0 .. pos(i); decode is Lq = 1 with the new token at Lkv - 1).
+ *   0 .. pos(i); decode is Lq = 1 with the new token at Lkv - 1, or at
+ *   kv_len[b] - 1 in hysparse_block_varlen / hysparse_block_paged).
  *
  * Layouts (row-major, contiguous, every pointer 16-byte aligned):
  *   q, q_sparse[n], out, out_sparse[n]  [B][Lq][Hq][d]   (dtype of the shape)
@@ -54,11 +55,13 @@ typedef struct CUstream_st *hs_stream_t;
 
 typedef enum {
     HS_OK = 0,
-    HS_ERR_INVALID_ARG = 1,   /* null or misaligned pointer, bad size, bad shape */
+    HS_ERR_INVALID_ARG = 1,   /* null or misaligned pointer, bad size, bad shape; (device) a
+                                 cache length outside [1, Lkv] (mixed-length / paged decode) */
     HS_ERR_UNSUPPORTED = 2,   /* valid but not implemented (dtype/d combination) */
     HS_ERR_WORKSPACE = 3,     /* ws_bytes below hysparse_workspace_size() */
     HS_ERR_CUDA = 4,          /* a CUDA call or kernel launch failed */
-    HS_ERR_INVALID_INDEX = 5, /* (device) an index list entry outside [-1, pos] */
+    HS_ERR_INVALID_INDEX = 5, /* (device) an index list entry outside [-1, pos], or a block
+                                 table entry outside the page pool (paged decode) */
     HS_ERR_TIMEOUT = 6        /* (device) a bounded wait inside a kernel gave up */
 } hs_status;
 
