@@ -431,10 +431,12 @@ __global__ void __launch_bounds__(SpSmem<NB>::SW * 32, 1) decode_full_mma(const 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long item = (long long)blockIdx.x * SpSmem<NB>::SW + warp;
     if (item >= (long long)p.B * p.Hkv * dp.nchunk) return;
-    const int ch = (int)(item % dp.nchunk);
-    const long long bg = item / dp.nchunk;
-    const int g = (int)(bg % p.Hkv);
-    const int b = (int)(bg / p.Hkv);
+    // KV head fastest: neighbouring warps read the same keys' adjacent
+    // 256-byte head slices of each 2 KB K and V row
+    const int g = (int)(item % p.Hkv);
+    const long long rest = item / p.Hkv;
+    const int ch = (int)(rest % dp.nchunk);
+    const int b = (int)(rest / dp.nchunk);
     const int G = p.G;
     uint8_t *wbase = smem + warp * SpSmem<NB>::WARP_BYTES;
     uint8_t *qs = wbase + SpSmem<NB>::ST * STAGE_BYTES;
