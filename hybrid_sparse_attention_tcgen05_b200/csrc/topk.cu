@@ -359,6 +359,175 @@ __device__ __forceinline__ unsigned int wk_find(const unsigned int *h, unsigned 
     return (unsigned int)(32 * c + e);
 }
 
+// Once a digit pass has found the k-th key's bin, the keys above the bin
+// ("definites") are final and the few keys inside it ("candidates") can be
+// ranked among themselves: one pass over the row writes the definites in key
+// order, as the plain compaction does, and lists the candidates in the
+// warp's histogram space with their bits of y below the bin and the number
+// of definites before them.  The `remaining` candidates with the smallest
+// such bits (ties to the lower key) are then merged into the index list.
+// This replaces a second digit pass and the compaction (two passes over the
+// row) with one.
+constexpr int WK_CAND = WK_BINS / 2;     // key index + packed word each
+constexpr int WK_CAND_SHIFT = 19;        // bits of y below the bin kept per candidate
+constexpr int WK_DEF_BITS = 13;          // definites before it (topk < 8192)
+constexpr int WK_MOVE = 8;               // 32-entry chunks per batch of the final merge
+constexpr int WK_CAND_MIN_ROW = 6;       // rows of at least this many times topk keys (the merge costs
+                                         // about one pass over topk entries)
+static_assert(WK_CAND_SHIFT + WK_DEF_BITS == 32, "candidate word");
+
+template <bool AL>
+__device__ __forceinline__ void select_with_candidates(const unsigned int *u, int n4, int nt, unsigned int M,
+                                                       unsigned int pre, int sh, unsigned int R, int topk,
+                                                       unsigned int *h, int32_t *o, uint32_t *mrow, int W,
+                                                       int lane) {
+    unsigned int *ck = h, *cw = h + WK_CAND;
+    const unsigned int lt = (1u << lane) - 1u, lowm = (1u << sh) - 1u;
+    int base = 0, cb = 0;
+    for (int g0 = 0; g0 < n4 + 1; g0 += 32) {   // the extra step carries the tail keys
+        const int g = g0 + lane;
+        unsigned int x[4];
+        bool ok[4];
+        if (g < n4) {
+            const uint4 v = ld4<AL>(u, g);
+            x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+            ok[0] = ok[1] = ok[2] = ok[3] = true;
+        } else {
+            const int tail0 = 4 * n4 + 4 * (g - n4);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                ok[c] = g == n4 && c < nt;
+                x[c] = ok[c] ? __ldg(u + tail0 + c) : 0u;
+            }
+        }
+        // keys above M (a sampled maximum) lie above the bin
+        bool df[4], cd[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const unsigned int hi = (M - x[c]) >> sh;
+            df[c] = ok[c] && (x[c] > M || hi < pre);
+            cd[c] = ok[c] && x[c] <= M && hi == pre;
+        }
+        int before = 0, tot = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const unsigned int bb = __ballot_sync(FULL, df[c]);
+            before += __popc(bb & lt);
+            tot += __popc(bb);
+        }
+        int cbef = 0, ctot = 0;
+        const bool any_cd = __any_sync(FULL, cd[0] || cd[1] || cd[2] || cd[3]);
+        if (any_cd) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const unsigned int bb = __ballot_sync(FULL, cd[c]);
+                cbef += __popc(bb & lt);
+                ctot += __popc(bb);
+            }
+        }
+        int at = base + before, ca = cb + cbef;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (df[c] && at < topk) o[at] = 4 * g + c;
+            if (cd[c] && ca < WK_CAND) {
+                ck[ca] = (unsigned int)(4 * g + c);
+                cw[ca] = (((M - x[c]) & lowm) << WK_DEF_BITS) | (unsigned int)min(at, topk);
+            }
+            at += df[c];
+            ca += cd[c];
+        }
+        base += tot;
+        cb += ctot;
+        if (mrow) {   // definites' bits; the chosen candidates' are OR-ed in below
+            unsigned int wd = ((df[0] ? 1u : 0u) | (df[1] ? 2u : 0u) | (df[2] ? 4u : 0u) | (df[3] ? 8u : 0u))
+                              << (4 * (lane & 7));
+            wd |= __shfl_xor_sync(FULL, wd, 1);
+            wd |= __shfl_xor_sync(FULL, wd, 2);
+            wd |= __shfl_xor_sync(FULL, wd, 4);
+            const int w = g0 / 8 + (lane >> 3);
+            if ((lane & 7) == 0 && w < W) mrow[w] = wd;
+        }
+    }
+    if (mrow)   // words past the row's causal end
+        for (int w = 4 * ((n4 + 32) / 32) + lane; w < W; w += 32) mrow[w] = 0u;
+    __syncwarp();
+
+    // the R-th smallest candidate bits, bit by bit from the top: `ans` keeps
+    // the largest value with fewer than R candidates below it
+    const int C = min(cb, WK_CAND);
+    unsigned int ans = 0;
+    for (int bit = sh - 1; bit >= 0; --bit) {
+        const unsigned int t = ans | (1u << bit);
+        unsigned int c = 0;
+        for (int j = lane; j < C; j += 32) c += (cw[j] >> WK_DEF_BITS) < t;
+        if (__reduce_add_sync(FULL, c) < R) ans = t;
+    }
+    unsigned int nl = 0;
+    for (int j = lane; j < C; j += 32) nl += (cw[j] >> WK_DEF_BITS) < ans;
+    const int take_eq = (int)R - (int)__reduce_add_sync(FULL, nl);
+
+    // keep the chosen candidates (in key order, in place): key, definites before it
+    int sb = 0, eb = 0;
+    for (int j0 = 0; j0 < C; j0 += 32) {
+        const int j = j0 + lane;
+        const bool v = j < C;
+        const unsigned int key = v ? ck[j] : 0u, wv = v ? cw[j] : 0u;
+        const unsigned int low = wv >> WK_DEF_BITS;
+        const bool eq = v && low == ans;
+        const unsigned int eqb = __ballot_sync(FULL, eq);
+        const bool sel = v && (low < ans || (eq && eb + __popc(eqb & lt) < take_eq));
+        eb += __popc(eqb);
+        const unsigned int sbb = __ballot_sync(FULL, sel);
+        __syncwarp();
+        if (sel) {
+            const int p = sb + __popc(sbb & lt);
+            ck[p] = key;
+            cw[p] = wv & ((1u << WK_DEF_BITS) - 1u);
+            if (mrow) atomicOr(mrow + (key >> 5), 1u << (key & 31u));
+        }
+        sb += __popc(sbb);
+        __syncwarp();
+    }
+
+    // definite d moves up by the number of chosen candidates with at most d
+    // definites before them; from the top down, WK_MOVE chunks of 32 read
+    // before any is written, so no entry is overwritten before it is read
+    const int D = min(base, topk);
+    int jh = sb;
+    for (int t0 = (D - 1) & ~31; t0 >= 0 && jh > 0; t0 -= 32 * WK_MOVE) {
+        int key[WK_MOVE], rs[WK_MOVE];
+#pragma unroll
+        for (int q = 0; q < WK_MOVE; ++q) {
+            const int d0 = t0 - 32 * q, d = d0 + lane;
+            rs[q] = 0;
+            key[q] = 0;
+            if (d0 < 0 || jh == 0) continue;
+            while (jh > 0 && (int)cw[jh - 1] > d0 + 31) --jh;
+            int k = jh, cnt = 0;
+            while (k > 0) {
+                const int db = (int)cw[k - 1];
+                if (db < d0) break;
+                cnt += db <= d;
+                --k;
+            }
+            rs[q] = d < D ? k + cnt : 0;
+            if (rs[q] > 0) key[q] = __ldcg(o + d);
+            jh = k;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < WK_MOVE; ++q) {
+            const int d = t0 - 32 * q + lane;
+            if (rs[q] > 0 && d + rs[q] < topk) o[d + rs[q]] = key[q];
+        }
+    }
+    __syncwarp();
+    for (int j = lane; j < sb; j += 32) {
+        const int p = j + (int)cw[j];
+        if (p < topk) o[p] = (int)ck[j];
+    }
+}
+
 template <bool AL>
 __global__ void __launch_bounds__(WK_WARPS * 32, 5)
 topk_warp_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv, int Hkv, int row_begin,
@@ -459,6 +628,13 @@ topk_warp_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv
     }
 
     while (top > 0) {
+        // After a digit pass that left few keys in the k-th key's bin, settle
+        // the rest from those keys alone (one more pass over the row, not two)
+        if (hs_ < 32 && top <= WK_CAND_SHIFT && cnt_eq <= (unsigned int)WK_CAND && topk < (1 << WK_DEF_BITS) &&
+            n >= WK_CAND_MIN_ROW * topk) {
+            select_with_candidates<AL>(u, n4, nt, M, pre, hs_, remaining, topk, h, o, mrow, W, lane);
+            return;
+        }
         const int s = max(0, top - WK_BITS);
         const unsigned int msk = (1u << (top - s)) - 1u;
         if (hs_ >= 32) {

@@ -131,7 +131,8 @@ TOPK_BUCKET_EDGES = (9984, 25600)
 
 @pytest.mark.parametrize("case", ["ties", "ties_unaligned", "all_equal", "zeros_and_denormals", "long_rows",
                                   "flat_narrow", "flat_long_unaligned", "many_rows_ties",
-                                  "many_rows_ties_aligned", "rows_8192", "short_rows_between_long"]
+                                  "many_rows_ties_aligned", "rows_8192", "short_rows_between_long",
+                                  "clustered", "clustered_wide"]
                          + [f"edge{e}" for e in TOPK_BUCKET_EDGES]
                          + [f"edge{e}_unaligned" for e in TOPK_BUCKET_EDGES])
 @pytest.mark.parametrize("kernel", ["block", "warp"])
@@ -161,6 +162,8 @@ def test_topk_synthetic_rows_bit_exact(case, kernel, monkeypatch):
         B, Hkv, Lq, Lkv, k = 1, 2, 300, 8192, 1000
     elif case == "short_rows_between_long":   # rows with n <= k end every (b, g) block
         B, Hkv, Lq, Lkv, k = 2, 2, 1500, 1500, 700
+    elif case.startswith("clustered"):   # the k-th key's bin holds more keys than the candidate list
+        B, Hkv, Lq, Lkv, k = 1, 2, 2100, 3000, 900
     s = torch.rand(B, Hkv, Lq, Lkv, generator=g)
     if case in ("ties", "ties_unaligned"):
         s = torch.round(s * 16) / 16
@@ -176,6 +179,11 @@ def test_topk_synthetic_rows_bit_exact(case, kernel, monkeypatch):
         s = torch.round(s * 65536) / 65536
     elif case.startswith("flat"):
         s = (1.0 + 0.02 * s) / 8192.0
+    elif case.startswith("clustered"):
+        # 80 % of the keys within 2^9 (2^14) fp32 steps above 0.5, the rest uniform
+        span = 2.0 ** (-15 if case == "clustered" else -10)
+        c = 0.5 + span * torch.rand(s.shape, generator=g)
+        s = torch.where(torch.rand(s.shape, generator=g) < 0.8, c, s)
     shape = hs.HsShape(B, Lq, Lkv, 4 * Hkv, Hkv, 128, 1, 0.0)
     idx = hs.topk(shape, s.to(DEV), k)
     n_valid = [Lkv - Lq + i + 1 for _ in range(B) for _ in range(Hkv) for i in range(Lq)]
