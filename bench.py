@@ -228,7 +228,9 @@ def bench_ours(args, w, ws_, rank, local):
     q, k, v = inp["q"], inp["k"], inp["v"]
     qs, gates = inp["q_sparse"], inp["gate"]
     shape = hs.shape_of(q, k)
-    chunk = args.row_chunk if args.row_chunk > 0 else min(w.Lq, max(1, (1 << 31) // (4 * w.Hkv * w.B * w.Lkv)))
+    # rows scored per chunk: an 8 GiB f32 score buffer (8192 rows at 32k and 64k keys) keeps the
+    # full layer's grids wide enough to fill the SMs (2 GiB chunks measured slower at both)
+    chunk = args.row_chunk if args.row_chunk > 0 else min(w.Lq, max(1, (1 << 33) // (4 * w.Hkv * w.B * w.Lkv)))
     chunk = min(chunk, w.Lq)
     n_chunks = math.ceil(w.Lq / chunk)
     out = torch.empty_like(q)

@@ -33,6 +33,7 @@
 // runs on the tensor cores while they are still turning S_j into P_j.
 // The running max is only moved when it grows by more than 8 (log2 units);
 // the final normalisation uses the same reference, so the result is exact.
+#include <algorithm>
 #include <cstring>
 
 #include <cuda.h>
@@ -482,6 +483,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 
 constexpr int SC_Q_STAGES = 4;   // Q slots: all G query tiles stay resident when G <= 4, else a ring
 constexpr int SC_K_STAGES = 2;
+constexpr int kScUnitsPerSm = 6;   // key-segment CTAs per SM a score launch aims for
+constexpr int kScMinSeg = 8;       // fewest key tiles per CTA (its Q tiles are loaded once per CTA)
 constexpr int SC_BUFS = 4;
 // warps 0-15 scores (four per TMEM lane quarter, 32 columns each), 16 TMA, 17 MMA
 constexpr int SC_SCORE_WARPS = 16;
@@ -513,6 +516,7 @@ struct ScParams {
     unsigned int *status;
     unsigned long long wait_ns;
     int tma_store;   // scores leave through `ts` (bulk tensor stores) rather than per-thread stores
+    int kv_seg;      // key tiles per CTA: blockIdx.x = segment * Hkv + KV head
 };
 
 __global__ void __launch_bounds__(SC_THREADS, 1)
@@ -530,12 +534,18 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     tile_of_block((p.row_end - p.row_begin + BM - 1) / BM, tile, b);   // heaviest row tiles first
     const int r0 = p.row_begin + tile * BM;
     const int r_end = min(r0 + BM, p.row_end);
-    const int g = blockIdx.x;
+    // The scores of different keys are independent once the forward pass has
+    // saved each row's statistics, so a row tile's causal key range is split
+    // into segments of kv_seg tiles, one CTA each: the grid fills the SMs
+    // even when a row chunk has few row tiles.
+    const int g = blockIdx.x % p.Hkv;
+    const int j_begin = (blockIdx.x / p.Hkv) * p.kv_seg;
     const int G = p.G;
     const bool resident = G <= SC_Q_STAGES;
     const int off = p.Lkv - p.Lq;
     const int pos_last = off + r_end - 1;
-    const int n_kv = pos_last / BN + 1;
+    if (j_begin > pos_last / BN) return;   // segment past this row tile's causal end: nothing set up yet
+    const int n_kv = min(pos_last / BN + 1 - j_begin, p.kv_seg);   // key tiles j_begin .. j_begin + n_kv - 1
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SC_Q_STAGES; ++s) {
@@ -584,7 +594,7 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 const uint32_t kb = smem_u32(&bars->k_full[sk_]);
                 mbar_expect_tx(kb, TILE);
                 for (int hf = 0; hf < 2; ++hf)
-                    tma_load_4d(smem_u32(sk + sk_ * TILE + hf * HALF), &tk, kb, hf * 64, g, j * BN, b);
+                    tma_load_4d(smem_u32(sk + sk_ * TILE + hf * HALF), &tk, kb, hf * 64, g, (j_begin + j) * BN, b);
                 k_issued = j + 1;
                 for (int hh = 0; !resident && hh < G; ++hh) {
                     const int it = j * G + hh, sq_ = it % SC_Q_STAGES;
@@ -680,7 +690,7 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 }
             }
             if (!ok) break;
-            const int j0 = j * BN + 32 * cq;
+            const int j0 = (j_begin + j) * BN + 32 * cq;
             const int keep = pos - j0 + 1;                  // causal columns of this row in the 32
             if (p.tma_store) {
                 // 2 boxes of 32 rows x 16 columns through the staging buffer
@@ -758,6 +768,19 @@ static cudaError_t fwd_prepare() {
     return a.numRegs == kFwdLaunchRegs ? cudaSuccess : cudaErrorInvalidDeviceFunction;
 }
 
+// SMs of the current device, read once per device.
+static int num_sms() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void *k, const void *v,
                                        void *out, float *lse, float *scores, long long ld,
                                        int row_begin, int row_count, float2 *stats,
@@ -786,7 +809,24 @@ cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || scores == nullptr) return e;
     ScParams sp{s.Lq, s.Lkv, s.Hq, s.Hkv, s.G(), row_begin, row_begin + row_count, row_count,
-                s.scale * kLog2e, stats, scores, ld, status, wait_ns, 0};
+                s.scale * kLog2e, stats, scores, ld, status, wait_ns, 0, 0};
+    // One CTA per (row tile, KV head) while the heaviest row tile is well
+    // under an SM's share of the chunk's causal (row tile, key tile) pairs;
+    // otherwise key segments, about kScUnitsPerSm CTAs per SM of at least
+    // kScMinSeg key tiles each (measured: splitting a grid that is already
+    // balanced costs a few percent in Q reloads and CTA start-up).
+    const long long off = (long long)s.Lkv - s.Lq;
+    long long pairs = 0;
+    for (int t = 0; t < n_tiles; ++t)
+        pairs += (off + min(row_begin + (t + 1) * BM, row_begin + row_count) - 1) / BN + 1;
+    const long long total = pairs * s.Hkv * s.B;
+    const int n_kv_max = (int)((off + row_begin + row_count - 1) / BN + 1);
+    sp.kv_seg = n_kv_max;
+    if (3ll * n_kv_max * num_sms() > 2 * total) {
+        const long long units = (long long)kScUnitsPerSm * num_sms();
+        sp.kv_seg = (int)std::min<long long>(n_kv_max, std::max<long long>(kScMinSeg, (total + units - 1) / units));
+    }
+    const int n_seg = (n_kv_max + sp.kv_seg - 1) / sp.kv_seg;
     // scores [B][Hkv][row_count][ld] f32 as a 3-D map (key, row, batch*KV head)
     // with 16 x 32 boxes in the 64-byte swizzle; needs 16-byte aligned rows
     CUtensorMap ms;
@@ -802,7 +842,7 @@ cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
             sp.tma_store = 1;
     }
-    attn_scores_tc<<<tile_grid(s.Hkv, n_tiles, s.B), SC_THREADS, kScSmem, st>>>(mq, mk, ms, sp); count_launch();
+    attn_scores_tc<<<tile_grid(s.Hkv * n_seg, n_tiles, s.B), SC_THREADS, kScSmem, st>>>(mq, mk, ms, sp); count_launch();
     return cudaGetLastError();
 }
 
