@@ -310,7 +310,9 @@ topk_radix_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lk
 // work (histogram scans, clears) is one warp's and no block barrier is
 // needed; the compaction runs once over the row in key order (ballots give
 // each selected key its output slot), with no separate counting pass.  The
-// row is re-read from global memory (L1 / L2) by each of its passes.
+// row is re-read from global memory (L1 / L2) by each of its passes: three
+// (sampled first digit, second digit, compaction), or two for long rows,
+// whose compaction also settles the k-th key's bin (select_with_candidates).
 
 constexpr int WK_WARPS = 8;
 constexpr int WK_BITS = 10;
