@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -134,12 +135,22 @@ class ClockSampler:
                 "reasons": names, "samples": len(self.samples)}
 
 
+def code_only(text: str) -> str:
+    """Source text without comments and blank lines, so that a recorded
+    measurement of a kernel survives edits to its comments."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (ln.split("//", 1)[0].rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln.strip())
+
+
 def source_hash(*names):
+    """sha1 (12 hex digits) of the named kernel sources' code, comments and
+    blank lines left out."""
     h = hashlib.sha1()
     for n in names:
         p = os.path.join(ROOT, "hybrid_sparse_attention_tcgen05_b200", "csrc", n)
         if os.path.exists(p):
-            h.update(open(p, "rb").read())
+            h.update(code_only(open(p, encoding="utf-8").read()).encode())
     return h.hexdigest()[:12]
 
 
