@@ -29,7 +29,9 @@
  * Conventions for every entry point:
  *   - All device buffers are owned by the caller (e.g. allocated by PyTorch).
  *     The library allocates no device or host memory and keeps no state
- *     between calls; scratch lives in the caller's workspace `ws`.
+ *     between calls beyond one-time kernel attributes and each device's SM
+ *     count (read once, to size grids); scratch lives in the caller's
+ *     workspace `ws`.
  *   - Work is enqueued on `stream` and is asynchronous; nothing synchronises
  *     except hysparse_workspace_status.
  *   - Arguments are checked on the host before anything is launched; a
