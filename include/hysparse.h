@@ -41,6 +41,10 @@
  *     d = 128; Hq % Hkv == 0; 1 <= Hq / Hkv <= 32; Lq <= Lkv;
  *     1 <= topk <= 4096; 1 <= window <= 1024.
  *   - NaN or Inf inputs give undefined (but memory-safe) results.
+ *   - One GPU per process: each kernel's one-time set-up (its shared-memory
+ *     attribute) runs on the first call, on that call's device, and is not
+ *     guarded against a concurrent first call; make the first call of each
+ *     kind from one host thread.  Later calls may come from any thread.
  */
 #ifndef HYSPARSE_H
 #define HYSPARSE_H
