@@ -33,7 +33,6 @@ EXPORTS = (
     "hysparse_block_paged",
     "hysparse_full_attn_scores_noalloc",
     "hysparse_workspace_status",
-    "hysparse_selftest_exp2",
     "hysparse_launch_count",
     "hysparse_status_string",
     "hysparse_version",
@@ -83,8 +82,6 @@ def lib():
     L.hysparse_block_paged.restype = I
     L.hysparse_full_attn_scores_noalloc.argtypes = [SP, P, P, P, P, P, P, LL, I, I, P]
     L.hysparse_full_attn_scores_noalloc.restype = I
-    L.hysparse_selftest_exp2.argtypes = [P, P, P, I, P]
-    L.hysparse_selftest_exp2.restype = I
     L.hysparse_launch_count.argtypes = []
     L.hysparse_launch_count.restype = ctypes.c_ulonglong
     L.hysparse_workspace_status.argtypes = [P, P]

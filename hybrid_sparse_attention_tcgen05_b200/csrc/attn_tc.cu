@@ -49,15 +49,6 @@ namespace hs {
 namespace tc {
 namespace {
 
-// Share of the softmax exponentials computed by exp2_poly on the FMA pipe
-// instead of the MUFU unit: every kFwdPolyEvery-th element of the forward
-// pass, every kScPolyEvery-th of the score pass (0 = none).  Measured on
-// B200 with the packed f32x2 FMAs: both passes are fastest with every
-// exponential on the MUFU unit (the polynomial's instructions cost more
-// issue slots than the MUFU time they free).
-constexpr int kFwdPolyEvery = 0;
-constexpr int kScPolyEvery = 0;
-
 constexpr int FWD_KV = 3;   // K/V ring slots (shared memory also holds Q0, Q1, P0, P1)
 
 struct FwdBars {
@@ -348,7 +339,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                 for (int e = 0; e < 4; ++e) {
                     const int c = ch * 8 + 2 * e;
                     const float2 t = ffma2(make_float2(s[c], s[c + 1]), c2v, mv);
-                    const float2 ab = make_float2(ex2_mix<kFwdPolyEvery>(t.x, c), ex2_mix<kFwdPolyEvery>(t.y, c + 1));
+                    const float2 ab = make_float2(ex2(t.x), ex2(t.y));
                     if (e & 1) ps23 = fadd2(ps23, ab); else ps01 = fadd2(ps01, ab);
                     pk[e] = pack_bf16(ab.x, ab.y);
                 }
@@ -392,6 +383,11 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                 p.lse[si] = (m + log2f(l)) * kLn2;
                 if (p.stats) p.stats[si] = make_float2(m, inv_l);
             }
+        }
+        if (!fin && MODE == FWD_FULL && valid) {
+            // a bounded wait gave up: mark the row's LSE, which callers own,
+            // so that the timeout is visible without the workspace status word
+            p.lse[((size_t)b * p.Hq + h0 + w) * p.Lq + row] = __int_as_float(0x7fc00000);
         }
         if (fin && MODE == FWD_WIN) {
             // normalised window branch, bf16 (the precision of the branch
@@ -515,6 +511,7 @@ struct ScParams {
     long long ld;
     unsigned int *status;
     unsigned long long wait_ns;
+    float *lse;      // [B][Hq][Lq]: set to NaN for this tile's rows and heads if a wait gives up
     int tma_store;   // scores leave through `ts` (bulk tensor stores) rather than per-thread stores
     int kv_seg;      // key tiles per CTA: blockIdx.x = segment * Hkv + KV head
 };
@@ -683,7 +680,7 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
                     const float2 t = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), c2v, mv);
-                    const float2 e = make_float2(ex2_mix<kScPolyEvery>(t.x, c), ex2_mix<kScPolyEvery>(t.y, c + 1));
+                    const float2 e = make_float2(ex2(t.x), ex2(t.y));
                     const float2 a2 = ffma2(e, lv, make_float2(acc[c], acc[c + 1]));
                     acc[c] = a2.x;
                     acc[c + 1] = a2.y;
@@ -741,7 +738,15 @@ attn_scores_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
-    if (threadIdx.x == 0 && bars->abort) report(p.status, HS_ERR_TIMEOUT);
+    if (bars->abort) {
+        // a bounded wait gave up: this tile's scores are undefined; mark the
+        // LSE of its rows and heads (caller-owned) so that the timeout is visible
+        for (int e = threadIdx.x; e < G * BM; e += blockDim.x) {
+            const int row = r0 + (e & (BM - 1));
+            if (row < r_end) p.lse[((size_t)b * p.Hq + g * G + (e >> 7)) * p.Lq + row] = __int_as_float(0x7fc00000);
+        }
+        if (threadIdx.x == 0) report(p.status, HS_ERR_TIMEOUT);
+    }
 }
 
 // ----------------------------------------------------------------- host side
@@ -809,7 +814,7 @@ cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || scores == nullptr) return e;
     ScParams sp{s.Lq, s.Lkv, s.Hq, s.Hkv, s.G(), row_begin, row_begin + row_count, row_count,
-                s.scale * kLog2e, stats, scores, ld, status, wait_ns, 0, 0};
+                s.scale * kLog2e, stats, scores, ld, status, wait_ns, lse, 0, 0};
     // One CTA per (row tile, KV head) while the heaviest row tile is well
     // under an SM's share of the chunk's causal (row tile, key tile) pairs;
     // otherwise key segments, about kScUnitsPerSm CTAs per SM of at least
@@ -883,21 +888,5 @@ cudaError_t sparse_pair_tc_launch(const Shape &s, const void *q, const void *k, 
     return cudaGetLastError();
 }
 
-namespace {
-__global__ void selftest_exp2_kernel(const float *x, float *yp, float *ym, int n) {
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < n) {
-        yp[i] = tc::exp2_poly(x[i]);
-        ym[i] = tc::ex2(x[i]);
-    }
-}
-}  // namespace
 
 }  // namespace hs
-
-extern "C" int hysparse_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int n, hs_stream_t stream) {
-    if (n < 0 || (n > 0 && (x == nullptr || y_poly == nullptr || y_mufu == nullptr))) return HS_ERR_INVALID_ARG;
-    if (n == 0) return HS_OK;
-    hs::selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, (cudaStream_t)stream>>>(x, y_poly, y_mufu, n); hs::count_launch();
-    return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
-}

@@ -81,37 +81,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-// 2^x on the FMA/ALU pipes, to take part of the exponentials off the MUFU
-// unit.  Cody-Waite-style range reduction x = n + f with n = rint(x) (by the
-// 1.5*2^23 addition trick) and f in [-1/2, 1/2]; 2^f by a degree-5
-// polynomial fitted by the Remez exchange algorithm on the relative error
-// (fit_exp2.py prints these coefficients); 2^n is added to the exponent
-// field.  Relative error <= 2.2e-7 (1.8 ulp) in fp32 for x >= -125; x < -125
-// (including -inf) gives 0.
-__device__ __forceinline__ float exp2_poly(float x) {
-    const float xc = fmaxf(x, -125.0f);
-    const float t = xc + 12582912.0f;            // 1.5 * 2^23: rounds xc to an integer
-    const float n = t - 12582912.0f;
-    const float f = xc - n;
-    float p = 1.327647245e-03f;
-    p = fmaf(p, f, 9.675540961e-03f);
-    p = fmaf(p, f, 5.550713092e-02f);
-    p = fmaf(p, f, 2.402212024e-01f);
-    p = fmaf(p, f, 6.931469440e-01f);
-    p = fmaf(p, f, 1.000000119e+00f);
-    const int ni = __float_as_int(t) - 0x4B400000;
-    const float r = __int_as_float(__float_as_int(p) + (ni << 23));
-    return x < -125.0f ? 0.0f : r;
-}
-
-// Element c of an unrolled softmax loop: every EVERY-th element takes the
-// polynomial (FMA pipe), the others the MUFU ex2 (EVERY = 0: all MUFU).
-template <int EVERY>
-__device__ __forceinline__ float ex2_mix(float x, int c) {
-    if (EVERY > 0 && (c % (EVERY > 0 ? EVERY : 1)) == EVERY - 1) return exp2_poly(x);
-    return ex2(x);
-}
-
 // Row-tile grids are launched as (heads, row tiles x batch): the hardware
 // hands out blocks in linear order with x fastest, so the heaviest causal
 // row tile of every head and batch is dispatched before any lighter one.

@@ -101,7 +101,10 @@ size_t hysparse_workspace_size(const hs_shape *shape, int topk, int window, int 
  *                              for j <= pos(i); entries j > pos(i) are left
  *                              unspecified and are never read by hysparse_topk.
  * `scores` may be NULL (forward pass only); otherwise ld_scores >= Lkv.
- * Only out/lse entries of the listed rows are written.
+ * Only out/lse entries of the listed rows are written.  If a bounded wait
+ * inside a kernel gives up (HS_ERR_TIMEOUT in the status word), the lse
+ * entries of the rows and heads it could not finish are set to NaN and their
+ * out and scores entries are undefined.
  * Decode (Lq == 1) uses split-K over the cache and needs `ws`.
  * Errors: HS_ERR_INVALID_ARG, HS_ERR_UNSUPPORTED, HS_ERR_WORKSPACE, HS_ERR_CUDA. */
 int hysparse_full_attn_scores(const hs_shape *shape, const void *q, const void *k, const void *v,
@@ -195,25 +198,34 @@ int hysparse_block_paged(const hs_shape *shape, const int32_t *kv_len, const int
 
 /* Allocation-free variant of hysparse_full_attn_scores (the pages have no
  * counterpart; this is a deployment convenience).  Same computation,
- * arguments, layouts and errors, but no workspace: its scratch (a status
- * word and the per-row softmax statistics, 256 + 8*B*Hq*Lq bytes rounded up
- * to 256) lives in a fixed 16 MiB device array inside the library, so callers
- * that may not allocate device memory -- a serving process that has frozen
- * its memory pool, or a plug-in host that only lends input and output
- * buffers -- can still run the full layer.  Every GPU that loads the library
- * holds that array until the process exits.
- *   - Shapes whose scratch exceeds 16 MiB return HS_ERR_WORKSPACE (score
- *     smaller row chunks or use hysparse_full_attn_scores instead).
+ * arguments, layouts and errors, but no workspace: its scratch lives in a
+ * fixed 16 MiB device array inside the library, so callers that may not
+ * allocate device memory -- a serving process that has frozen its memory
+ * pool, or a plug-in host that only lends input and output buffers -- can
+ * still run the full layer.  Every GPU that loads the library holds that
+ * array until the process exits.
+ *   - Scratch needed: 256 bytes (status word) + 8*B*Hq*Lq bytes of per-row
+ *     softmax statistics, rounded up to 256; decode-shaped calls (Lq == 1,
+ *     bf16) also keep their split-K partials and logit stash there, a
+ *     further 4*B*Hq*Lkv + 520*B*Hq*ceil(Lkv/1024) + 768 bytes rounded up
+ *     to 256.  Shapes needing more than 16 MiB return HS_ERR_WORKSPACE
+ *     before anything runs (score smaller row chunks, decode smaller
+ *     batches, or use hysparse_full_attn_scores).
  *   - Calls no cudaMalloc/cudaFree and allocates nothing; the caller still
  *     provides q, k, v, out, lse and (optionally) scores.
  *   - The array's device address is looked up on the first call on each
- *     device (the current device, which `stream` must belong to); make that
- *     first call before any stream capture.
+ *     device (the current device, which `stream` must belong to) and kept
+ *     for the life of the process; make that first call before any stream
+ *     capture, and do not use this entry point after cudaDeviceReset in the
+ *     same process (the array may move).
  *   - All calls share the one array and each zeroes its status word on
  *     `stream`: calls that can overlap on the GPU (other streams, other host
  *     threads without ordering) race on it and must be serialised by the
- *     caller.  Device-side timeouts are recorded there but are not readable
- *     through this API. */
+ *     caller.
+ *   - The status word cannot be read through this API.  A bounded wait that
+ *     gives up inside a tensor-core kernel (HS_ERR_TIMEOUT elsewhere) leaves
+ *     NaN in the lse entries of the rows and heads it could not finish; the
+ *     out and scores entries of those rows are then undefined. */
 int hysparse_full_attn_scores_noalloc(const hs_shape *shape, const void *q, const void *k,
                                       const void *v, void *out, float *lse, float *scores,
                                       long long ld_scores, int row_begin, int row_count,
@@ -223,12 +235,6 @@ int hysparse_full_attn_scores_noalloc(const hs_shape *shape, const void *q, cons
  * lowest-numbered device error recorded since it was last cleared), clears
  * it and returns it.  Returns HS_ERR_CUDA if the synchronisation fails. */
 int hysparse_workspace_status(void *ws, hs_stream_t stream);
-
-/* Diagnostic: y_poly[i] = the kernels' polynomial 2^x (FMA-pipe
- * exponential used for part of the softmax elements) and y_mufu[i] = the
- * hardware ex2 approximation, for n device floats x.  Lets a test check both
- * against exact 2^x.  Errors: HS_ERR_INVALID_ARG, HS_ERR_CUDA. */
-int hysparse_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int n, hs_stream_t stream);
 
 /* Diagnostic: number of CUDA kernels this library has launched in this
  * process so far (counted on the host at each launch). */

@@ -211,3 +211,60 @@ def test_binding_refuses_cpu_tensors(L):
     q = torch.zeros(1, 4, 4, 64)
     with pytest.raises(ValueError):
         hs.full_attn_scores(q, q[:, :, :1].contiguous(), q[:, :, :1].contiguous())
+
+
+NOALLOC_BYTES = 16 << 20
+
+
+def noalloc_scratch_bytes(B, Lq, Lkv, Hq, decode):
+    """Scratch of hysparse_full_attn_scores_noalloc as hysparse.h states it:
+    256 + 8*B*Hq*Lq rounded up to 256, plus for decode-shaped calls
+    4*B*Hq*Lkv + 520*B*Hq*ceil(Lkv/1024) + 768 rounded up to 256."""
+    up = lambda x: (x + 255) // 256 * 256
+    n = up(256 + 8 * B * Hq * Lq)
+    if decode:
+        n += up(4 * B * Hq * Lkv + 520 * B * Hq * ((Lkv + 1023) // 1024) + 768)
+    return n
+
+
+_NOALLOC_CHILD = r"""
+import ctypes, sys
+sys.path.insert(0, {root!r})
+from hybrid_sparse_attention_tcgen05_b200 import _lib
+L = _lib.lib()
+A = 0x7f0000000000
+P = lambda i: ctypes.c_void_p(A + (i << 32))
+for B, Lq, Lkv, Hq, Hkv in {cases!r}:
+    s = _lib.HsShape(B, Lq, Lkv, Hq, Hkv, 128, _lib.HS_BF16, 0.0)
+    print(L.hysparse_full_attn_scores_noalloc(ctypes.byref(s), P(1), P(2), P(3), P(4), P(5), None, 0, 0, Lq,
+                                              None))
+"""
+
+
+def test_noalloc_refuses_scratch_beyond_its_array():
+    """The size check of the allocation-free entry point comes before any
+    CUDA call.  Run in a child process that sees no GPU, so that a shape the
+    check lets through stops at the first CUDA call (HS_ERR_CUDA) instead of
+    launching anything on fake addresses.  Shapes on both sides of the 16 MiB
+    array, prefill- and decode-shaped, follow the bound hysparse.h states."""
+    import subprocess
+    import sys
+    cases = [(1, 65536, 65536, 64, 4),        # 8 B of statistics per (head, row): 32 MiB
+             (1, 32000, 32000, 64, 4),        # 16.0 MB: fits
+             (1, 32800, 32800, 64, 4),        # just over
+             (64, 1, 32768, 32, 8),           # the 64 x 32k decode step: its logit stash alone is 256 MiB
+             (2, 1, 1000, 8, 2),              # small decode: fits
+             (4, 1, 28000, 32, 8),            # decode just under the array
+             (4, 1, 30000, 32, 8)]            # and just over
+    expect = []
+    for B, Lq, Lkv, Hq, Hkv in cases:
+        n = noalloc_scratch_bytes(B, Lq, Lkv, Hq, Lq == 1)
+        expect.append(_lib.HS_ERR_WORKSPACE if n > NOALLOC_BYTES else _lib.HS_ERR_CUDA)
+    assert _lib.HS_ERR_WORKSPACE in expect and _lib.HS_ERR_CUDA in expect
+    hs_build.build()
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    res = subprocess.run([sys.executable, "-c", _NOALLOC_CHILD.format(root=ROOT, cases=cases)],
+                         capture_output=True, text=True, env=env, timeout=120)
+    assert res.returncode == 0, res.stderr
+    got = [int(x) for x in res.stdout.split()]
+    assert got == expect
