@@ -1,12 +1,16 @@
 """Benchmark of the HySparse hybrid block on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill8k]
-                    [--impl ours|reference] [--no-cpu-baseline]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload moe64k]
+                    [--impl ours|reference] [--no-cpu-baseline] [--no-decode]
+                    [--profile-stage full|topk|sparse]
 
 One step = one hybrid block over one batch of synthetic input: the full
 causal GQA layer with importance scores (row chunks), per-row top-k, then
 N sparse layers (global top-k branch + 128-token window + gate), each stage
-through the library's C ABI.  Prints ONE JSON line on rank 0.
+through the library's C ABI.  Prints ONE JSON line on rank 0.  The default
+workload is the largest single-GPU configuration (moe64k: 65536-token
+prefill, 64 query / 4 KV heads, 9 sparse layers); a prefill line also carries
+the decode step (64 sequences x 32768-token caches) under "decode".
 
 Multi-GPU: one process per GPU (torchrun).  Blocks are independent problems,
 so every rank runs its own replica of the workload with no collective on the
@@ -169,6 +173,35 @@ def read_traffic(kernel_key: str, src_hash: str):
     return None
 
 
+def measure_l2(dev, mb: int = 64, passes: int = 8, reps: int = 5):
+    """L2 read bandwidth on this GPU, measured live: the library's probe over
+    an L2-resident buffer of `mb` MiB (streaming 16-byte reads, and random
+    whole 256-byte rows as the sparse gather reads them), best of `reps`
+    timed calls after one untimed call that makes the buffer resident."""
+    import hybrid_sparse_attention_tcgen05_b200 as hs
+    props = torch.cuda.get_device_properties(dev)
+    blocks = props.multi_processor_count * 4
+    buf = torch.ones(mb << 20, dtype=torch.uint8, device=dev)
+    sink = torch.zeros(blocks, dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    out = {"buffer_mib": mb, "passes_per_call": passes, "blocks": blocks, "threads_per_block": 512}
+    for mode, key in ((0, "stream_gbs"), (1, "row_gather_gbs")):
+        hs.probe_l2_read(buf, 1, mode, blocks, sink)
+        best = 0.0
+        for _ in range(reps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            hs.probe_l2_read(buf, passes, mode, blocks, sink)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            best = max(best, passes * buf.numel() / (e0.elapsed_time(e1) / 1e3) / 1e9)
+        out[key] = best
+    out["peak_gbs"] = max(out["stream_gbs"], out["row_gather_gbs"])
+    del buf, sink
+    return out
+
+
 # ------------------------------------------------------------- work model
 
 def pairs_causal(w):
@@ -210,6 +243,17 @@ def work_model(w):
             "kv_bytes": kv_bytes, "keff": keff, "weff": weff, "pairs": P}
 
 
+# kernel sources of the gather sparse layer (their hash keys the traffic record)
+SPARSE_GATHER_SRCS = ("sparse_mma.cu", "sparse_gather_tc.cu", "tc_util.cuh")
+
+
+def l2_served(w):
+    """The gather reads one KV head's K and V at a time; when that slice
+    (B*Lkv*d*2 bytes each) fits comfortably in L2 its rows are L2 hits."""
+    esz = 2 if w.dtype == "bf16" else 4
+    return w.Lq > 1 and 2 * w.B * w.Lkv * w.d * esz <= 64 * 2 ** 20
+
+
 def sparse_path_is_dense(w):
     """The library's choice between the dense-masked and the gather sparse
     kernel (same estimate as hysparse_api.cu; HYSPARSE_SPARSE_PATH overrides)."""
@@ -235,6 +279,7 @@ def bench_ours(args, w, ws_, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks, peak_kind = load_peaks()
+    l2 = measure_l2(dev)
     inp = gen.make_inputs(w, seed=args.seed + rank, device=str(dev))
     q, k, v = inp["q"], inp["k"], inp["v"]
     qs, gates = inp["q_sparse"], inp["gate"]
@@ -477,11 +522,22 @@ def bench_ours(args, w, ws_, rank, local):
         launches = w.n_sparse
         dur_s = per["sparse"] / launches / 1e3
         achieved = wm["gather_bytes_per_layer"] / dur_s / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"kernel": "sparse_attn (gather: sparse_attn_mma)", "bound": "hbm", "unit": "GB/s",
+        if l2_served(w) and l2 is not None:
+            # one KV head's K and V fit in L2 and the kernel walks the items KV
+            # head by KV head: the gathered rows are L2 hits, rated against the
+            # measured L2 read bandwidth
+            peak = l2["peak_gbs"]
+            bound, peak_src = "l2", "measured L2 read bandwidth (library probe, this run)"
+        else:
+            peak = peaks["hbm_gbs"]
+            bound, peak_src = "hbm", None
+        roof = {"kernel": "sparse_attn (gather)", "bound": bound, "unit": "GB/s",
                 "work": "(k_eff + w_eff) K and V rows per (row, kv head) + q, gate, out, idx"}
-        key, srcs = "sparse_attn", ("sparse_mma.cu",)
-    roof.update({"achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} (burst)",
+        if peak_src:
+            roof["peak_source"] = peak_src
+        key, srcs = "sparse_attn", SPARSE_GATHER_SRCS
+    roof.update({"achieved": achieved, "peak": peak,
+                 "peak_kind": "measured (L2 probe)" if roof["bound"] == "l2" else f"{peak_kind} (burst)",
                  "frac": achieved / peak, "launch_ms": dur_s * 1e3,
                  "traffic": read_traffic(f"{w.name}/{key}", source_hash(*srcs))})
     stage_ctx = {
@@ -496,8 +552,14 @@ def bench_ours(args, w, ws_, rank, local):
         "topk": {"ms": per["topk"], "gbs": (wm["score_bytes"] / 2 + 4.0 * w.B * w.Hkv * w.Lq * w.topk)
                  / (per["topk"] / 1e3) / 1e9},
         "sparse_per_layer": {"ms": per["sparse"] / max(1, w.n_sparse),
+                             "path": "dense-masked" if sparse_dense else "gather",
                              "gbs": wm["gather_bytes_per_layer"] / (per["sparse"] / max(1, w.n_sparse) / 1e3) / 1e9},
     }
+    sp_gbs = stage_ctx["sparse_per_layer"]["gbs"]
+    if l2_served(w):
+        stage_ctx["sparse_per_layer"]["frac_of_l2"] = sp_gbs / l2["peak_gbs"]
+    else:
+        stage_ctx["sparse_per_layer"]["frac_of_hbm"] = sp_gbs / peaks["hbm_gbs"]
     res = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -517,6 +579,7 @@ def bench_ours(args, w, ws_, rank, local):
         "roofline": roof,
         "stages_ms_per_step": per,
         "stages": stage_ctx,
+        "l2_probe": l2,
         "wall_s_timed": wall,
     }
     if w.Lq == 1:
@@ -773,11 +836,12 @@ def bench_reference(args, w):
     per = args.cpu_budget / max(1, args.steps + args.warmup)
     for _ in range(args.warmup):
         oracle_sample_time(w, args.seed, per, host)
-    vals = []
+    vals, sample_s = [], []
     desc, threads = "", 1
     for _ in range(max(1, args.steps)):
-        e, desc, threads, _ = oracle_sample_time(w, args.seed, per, host)
+        e, desc, threads, ts = oracle_sample_time(w, args.seed, per, host)
         vals.append(e)
+        sample_s.append(ts)
     est = statistics.median(vals)
     tokens = w.B * w.Lq
     value = tokens / est
@@ -792,7 +856,62 @@ def bench_reference(args, w):
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        # each step times a row sample, not the whole workload: ms_per_step is
+        # the whole workload's time extrapolated from that sample
+        "extrapolated": True,
+        "sample_s_per_step": statistics.median(sample_s),
+        "sample_s_total": sum(sample_s),
     }
+
+
+def decode_summary(res, peaks):
+    """The decode step's figures for the headline line: step latency, tokens/s
+    (device and end to end), per-stage times, and the sparse gather stage's
+    achieved HBM bandwidth against the measured HBM peak."""
+    st = res["stages"]
+    sp = st["sparse_per_layer"]
+    return {"workload": res["config"]["workload"], "config": res["config"],
+            "decode_step_us": res["ms_per_step"] * 1e3, "value": res["value"], "unit": res["unit"],
+            "e2e": res["e2e"], "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
+            "stages_ms_per_step": res["stages_ms_per_step"],
+            "full": {"ms": st["full"]["ms"], "hbm_gbs": st["full"]["hbm_gbs"],
+                     "frac_of_hbm": st["full"]["hbm_gbs"] / peaks["hbm_gbs"]},
+            "sparse_gather": {"ms_per_layer": sp["ms"], "hbm_gbs": sp["gbs"],
+                              "frac_of_hbm": sp["gbs"] / peaks["hbm_gbs"], "peak_gbs": peaks["hbm_gbs"],
+                              "work": "(k_eff + w_eff) K and V rows per (sequence, kv head) + q, gate, "
+                                      "out, idx"},
+            "roofline": res["roofline"]}
+
+
+def profile_stage(args, w):
+    """A few launches of one stage on a small case, for ncu captures: the
+    inputs and the index set are made first (one untimed block), then the
+    stage's C-ABI call runs `--profile-reps` times."""
+    import hybrid_sparse_attention_tcgen05_b200 as hs
+    from hybrid_sparse_attention_tcgen05_b200 import inputs as gen
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = w.with_(n_sparse=1)
+    inp = gen.make_inputs(w, seed=args.seed, device=str(dev))
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    chunk = min(w.Lq, 4096)
+    out, lse, idx, outs = hs.block(q, k, v, inp["q_sparse"], inp["gate"], w.topk, w.window, row_chunk=chunk)
+    torch.cuda.synchronize()
+    shape = hs.shape_of(q, k)
+    ws = hs.alloc_workspace(shape, w.topk, w.window, 1, chunk, dev)
+    for _ in range(args.profile_reps):
+        if args.profile_stage == "sparse":
+            hs.sparse_attn(inp["q_sparse"][0], k, v, idx, inp["gate"][0], w.window, out=outs[0], ws=ws)
+        elif args.profile_stage == "full":
+            hs.full_attn_scores(q, k, v, row_begin=w.Lq - chunk, row_count=chunk, out=out, lse=lse, ws=ws)
+        else:
+            sc = hs.full_attn_scores(q, k, v, row_begin=w.Lq - chunk, row_count=chunk, out=out, lse=lse,
+                                     ws=ws)[2]
+            hs.topk(shape, sc, w.topk, row_begin=w.Lq - chunk, idx=idx)
+    torch.cuda.synchronize()
+    if hs.workspace_status(ws) != 0:
+        raise RuntimeError("device status set")
+    print(json.dumps({"profile_stage": args.profile_stage, "workload": w.name, "reps": args.profile_reps}))
 
 
 def main():
@@ -800,7 +919,13 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="prefill8k")
+    ap.add_argument("--workload", default="moe64k",
+                    help="headline workload (default: the largest single-GPU configuration)")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="prefill workloads: skip the decode step that the line also reports")
+    ap.add_argument("--profile-stage", choices=["full", "topk", "sparse"], default=None,
+                    help="run a few launches of one stage (for ncu) and exit; no timing")
+    ap.add_argument("--profile-reps", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--row-chunk", type=int, default=0)
@@ -819,6 +944,10 @@ def main():
     if args.seq > 0:
         w = w.with_(Lkv=args.seq, Lq=1 if w.Lq == 1 else args.seq, name=f"{w.name}@{args.seq}")
     world, rank, local = dist_env()
+
+    if args.profile_stage:
+        profile_stage(args, w)
+        return 0
 
     if args.impl == "reference":
         if rank != 0:
@@ -846,6 +975,14 @@ def main():
             res["cpu_baseline"] = {"value": w.B * w.Lq / est, "unit": "tokens/s", "cores": threads,
                                    "kind": "oracle", "sample": desc}
         res.pop("_inputs", None)
+        if w.Lq > 1 and not args.no_decode and args.seq == 0:
+            # the decode step of the same line (64 sequences, 32768-token caches)
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+            dres = bench_ours(args, gen.WORKLOADS["decode"], world, rank, local)
+            dres.pop("_inputs", None)
+            res["decode"] = decode_summary(dres, load_peaks()[0])
+            res["gpu_launches_decode"] = dres["gpu_launches"]
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

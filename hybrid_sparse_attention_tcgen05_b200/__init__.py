@@ -267,6 +267,17 @@ def workspace_status(ws: torch.Tensor) -> int:
     return int(_lib.lib().hysparse_workspace_status(_ptr(ws), _stream(dev)))
 
 
+def probe_l2_read(buf: torch.Tensor, passes: int, mode: int, blocks: int, sink: torch.Tensor) -> None:
+    """Enqueue one L2 read-bandwidth probe over the device buffer `buf`
+    (mode 0 streaming, 1 random 256-byte rows; passes * buf bytes read);
+    `sink` holds at least `blocks` int64 words.  Time it with CUDA events."""
+    dev = _need_cuda(buf, sink)
+    nbytes = buf.numel() * buf.element_size()
+    st = _lib.lib().hysparse_probe_l2_read(_ptr(buf), nbytes, int(passes), int(mode), int(blocks), _ptr(sink),
+                                           _stream(dev))
+    _lib.check(st, "hysparse_probe_l2_read")
+
+
 def launch_count() -> int:
     """Kernels launched by the library so far in this process."""
     return int(_lib.lib().hysparse_launch_count())

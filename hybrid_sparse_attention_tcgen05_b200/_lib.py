@@ -33,6 +33,7 @@ EXPORTS = (
     "hysparse_block_paged",
     "hysparse_full_attn_scores_noalloc",
     "hysparse_workspace_status",
+    "hysparse_probe_l2_read",
     "hysparse_launch_count",
     "hysparse_status_string",
     "hysparse_version",
@@ -82,6 +83,8 @@ def lib():
     L.hysparse_block_paged.restype = I
     L.hysparse_full_attn_scores_noalloc.argtypes = [SP, P, P, P, P, P, P, LL, I, I, P]
     L.hysparse_full_attn_scores_noalloc.restype = I
+    L.hysparse_probe_l2_read.argtypes = [P, SZ, I, I, I, P, P]
+    L.hysparse_probe_l2_read.restype = I
     L.hysparse_launch_count.argtypes = []
     L.hysparse_launch_count.restype = ctypes.c_ulonglong
     L.hysparse_workspace_status.argtypes = [P, P]

@@ -236,6 +236,22 @@ int hysparse_full_attn_scores_noalloc(const hs_shape *shape, const void *q, cons
  * it and returns it.  Returns HS_ERR_CUDA if the synchronisation fails. */
 int hysparse_workspace_status(void *ws, hs_stream_t stream);
 
+/* Diagnostic (no counterpart on the pages): L2 read bandwidth probe, the
+ * denominator for kernels whose reads are served from L2 (the prefill sparse
+ * layers gather K/V rows from a cache that fits in L2).  Reads the DEVICE
+ * buffer `buf` (`bytes`, a multiple of 256 and >= 4096, 256-byte aligned; the
+ * caller makes it L2-resident, e.g. by one untimed call first) with `blocks`
+ * CTAs of 512 threads on `stream`, using L2-only loads:
+ *   mode 0: streaming 16-byte reads, `passes` times over the buffer;
+ *   mode 1: whole 256-byte rows at hashed positions, passes * bytes / 256
+ *           rows (the access pattern of the sparse layers' row gather).
+ * Either way passes * bytes bytes are read; time the call with events on
+ * `stream`.  `sink` is a DEVICE array of at least `blocks` 64-bit words that
+ * receives an XOR of what each CTA read (it keeps the loads live).
+ * Errors: HS_ERR_INVALID_ARG, HS_ERR_CUDA. */
+int hysparse_probe_l2_read(const void *buf, size_t bytes, int passes, int mode, int blocks,
+                           unsigned long long *sink, hs_stream_t stream);
+
 /* Diagnostic: number of CUDA kernels this library has launched in this
  * process so far (counted on the host at each launch). */
 unsigned long long hysparse_launch_count(void);

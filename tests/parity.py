@@ -18,6 +18,14 @@ import torch
 import oracle
 
 OUT_TOL = {"f32": 1e-4, "bf16": 2e-2}
+# Per-row relative L2 error gate, beside the absolute one.  On the shifted
+# prefill workloads the outputs are ~1e-3 (nearly flat softmax over values of
+# std 1/sqrt(d)), so the absolute bound alone would pass zeros; a row's error
+# relative to its own norm does not.  bf16: the output's rounding (unit
+# roundoff 2^-8, ~2.3e-3 rms relative) plus P rounded to bf16 before the PV
+# product (~2.3e-3 rms relative of a random-sign sum) give ~3.3e-3; the gate
+# is 1e-2.  fp32: a few ulp per term, ~1e-6; the gate is 1e-4.
+REL_L2_TOL = {"f32": 1e-4, "bf16": 1e-2}
 SCORE_RTOL = 2e-5
 LSE_ATOL = 1e-4
 TIE_BAND = 1e-6
@@ -55,10 +63,32 @@ def rel_l2(a: torch.Tensor, b: torch.Tensor) -> float:
     return float((a - b).norm() / max(float(b.norm()), 1e-300))
 
 
-def check_out(name: str, got: torch.Tensor, ref: torch.Tensor, dtype: str) -> None:
+def row_rel_l2(got: torch.Tensor, ref: torch.Tensor) -> torch.Tensor:
+    """Relative L2 error of every leading-index row ([R, ...] -> [R]); rows
+    whose reference is exactly zero (an empty branch) give their absolute
+    error norm."""
+    a = got.double().cpu().reshape(got.shape[0], -1)
+    b = ref.double().cpu().reshape(ref.shape[0], -1)
+    nb = b.norm(dim=1)
+    return (a - b).norm(dim=1) / torch.where(nb > 0, nb, torch.ones_like(nb))
+
+
+WORST = {}
+
+
+def check_out(name: str, got: torch.Tensor, ref: torch.Tensor, dtype: str) -> float:
+    """max-abs error <= OUT_TOL (the contract's bound) and, per row, relative
+    L2 error <= REL_L2_TOL.  Returns the worst row's relative L2 error (also
+    kept in WORST under `name` and printed, so pytest -s shows it)."""
     err = max_abs(got, ref)
+    rel = float(row_rel_l2(got, ref).max()) if got.numel() else 0.0
+    WORST[name] = max(rel, WORST.get(name, 0.0))
+    print(f"[parity] {name}: max abs {err:.3e}, worst row rel L2 {rel:.3e}")
     tol = OUT_TOL[dtype]
-    assert err <= tol, f"{name}: max abs error {err:.3e} > {tol:.1e} (rel L2 {rel_l2(got, ref):.2e})"
+    assert err <= tol, f"{name}: max abs error {err:.3e} > {tol:.1e} (worst row rel L2 {rel:.2e})"
+    rtol = REL_L2_TOL[dtype]
+    assert rel <= rtol, f"{name}: worst row relative L2 error {rel:.3e} > {rtol:.0e} (max abs {err:.2e})"
+    return rel
 
 
 def check_topk(gpu_idx: torch.Tensor, ora_scores: torch.Tensor, n_valid: Sequence[int], topk: int) -> Dict[str, int]:

@@ -22,7 +22,7 @@ def test_zero_wait_limit_reports_timeout_and_context_survives():
     old = os.environ.get("HYSPARSE_WAIT_LIMIT_NS")
     os.environ["HYSPARSE_WAIT_LIMIT_NS"] = "0"
     try:
-        hs.full_attn_scores(inp["q"], inp["k"], inp["v"], ws=ws)
+        _, lse_to, _ = hs.full_attn_scores(inp["q"], inp["k"], inp["v"], ws=ws)
         st = hs.workspace_status(ws)
     finally:
         if old is None:
@@ -30,6 +30,7 @@ def test_zero_wait_limit_reports_timeout_and_context_survives():
         else:
             os.environ["HYSPARSE_WAIT_LIMIT_NS"] = old
     assert st == _lib.HS_ERR_TIMEOUT
+    assert torch.isnan(lse_to).any()      # the rows it gave up on are marked in the caller's lse
     # status word was cleared; a normal call now succeeds and reports OK
     out, lse, sc = hs.full_attn_scores(inp["q"], inp["k"], inp["v"], ws=ws)
     assert hs.workspace_status(ws) == _lib.HS_OK

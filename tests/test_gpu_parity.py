@@ -68,6 +68,29 @@ def oracle_check_rows(inp, w, rows, out, lse, idx, scores_all, outs, check_own_i
     return stats, o_idx
 
 
+def check_sparse_on_oracle_idx(inp, w, rows, idx, o_idx, tag=""):
+    """Run every sparse layer on the oracle's own index sets: the GPU index
+    tensor with the sampled rows replaced by the oracle's sets (o_idx
+    [nrows, Hkv, k]), one layer at a time, compared on those rows with the
+    oracle's sparse layer over the same sets."""
+    scale = scale_of(w.d)
+    k_h, v_h = inp["k"].to("cpu"), inp["v"].to("cpu")
+    b = torch.tensor([r[0] for r in rows], device=idx.device)
+    i = torch.tensor([r[1] for r in rows], device=idx.device)
+    idx_o = idx.clone()
+    idx_o[b, :, i] = o_idx.to(idx.device, torch.int32)
+    for n, (qs, gt) in enumerate(zip(inp["q_sparse"], inp["gate"])):
+        g_out, g_og, g_ol = hs.sparse_attn(qs, inp["k"], inp["v"], idx_o, gt, w.window, want_branches=True)
+        torch.cuda.synchronize()
+        r_out, r_og, r_ol = oracle.sparse_rows(gather_rows(qs, rows), k_h, v_h, rows, w.Lq, scale, o_idx,
+                                               gather_rows(gt, rows), w.window)
+        check_out(f"{tag}sparse{n} out (oracle idx)", gather_rows(g_out, rows), r_out, w.dtype)
+        check_out(f"{tag}sparse{n} global (oracle idx)", gather_rows(g_og, rows), r_og, w.dtype)
+        check_out(f"{tag}sparse{n} local (oracle idx)", gather_rows(g_ol, rows), r_ol, w.dtype)
+        del g_out, g_og, g_ol
+    del idx_o
+
+
 def sparse_on_indices(inp, w, idx_dev):
     return [hs.sparse_attn(qs, inp["k"], inp["v"], idx_dev, gt, w.window, want_branches=True)
             for qs, gt in zip(inp["q_sparse"], inp["gate"])]
@@ -324,7 +347,10 @@ def test_full_size_prefill_sampled_rows(name, sparse_path):
     n_rand = {"prefill8k": 96, "prefill32k": 48, "moe64k": 24}[name]
     rows = rows_for(w.B, w.Lq, gen.sample_rows(w.Lq, w.topk, w.window, n_random=n_rand, seed=0,
                                                edge=8))
-    oracle_check_rows(inp, w, rows, out, lse, idx, None, sp)
+    _, o_idx = oracle_check_rows(inp, w, rows, out, lse, idx, None, sp)
+    del sp, outs_list
+    # the same sparse kernels on the oracle's index sets for the sampled rows
+    check_sparse_on_oracle_idx(inp, w, rows, idx, o_idx, tag=f"{name}: ")
 
 
 def test_full_size_decode_sampled_batches():
@@ -335,10 +361,15 @@ def test_full_size_decode_sampled_batches():
     sp = [hs.sparse_attn(qs, inp["k"], inp["v"], idx, gt, w.window, want_branches=True)
           for qs, gt in zip(inp["q_sparse"], inp["gate"])]
     torch.cuda.synchronize()
-    for b in (0, 21, 42, 63):
+    picked = (0, 21, 42, 63)
+    o_sets = []
+    for b in picked:
         one = {"q": inp["q"][b:b + 1], "k": inp["k"][b:b + 1], "v": inp["v"][b:b + 1],
                "q_sparse": [x[b:b + 1] for x in inp["q_sparse"]],
                "gate": [x[b:b + 1] for x in inp["gate"]]}
         w1 = w.with_(B=1)
-        oracle_check_rows(one, w1, [(0, 0)], out[b:b + 1], lse[b:b + 1], idx[b:b + 1], None,
-                          [tuple(t[b:b + 1] for t in s) for s in sp])
+        _, o_idx = oracle_check_rows(one, w1, [(0, 0)], out[b:b + 1], lse[b:b + 1], idx[b:b + 1], None,
+                                     [tuple(t[b:b + 1] for t in s) for s in sp])
+        o_sets.append(o_idx[0])
+    # the decode sparse kernels on the oracle's index sets of those sequences
+    check_sparse_on_oracle_idx(inp, w, [(b, 0) for b in picked], idx, torch.stack(o_sets), tag="decode: ")
