@@ -147,6 +147,16 @@ bool prefer_dense_sparse(const Shape &s, int topk, int window) {
     return dense_s < gather_s;
 }
 
+// Which gather kernel runs the sparse layer: the tcgen05 row gather
+// (sparse_gather_tc.cu) or the warp-MMA one (sparse_mma.cu).
+// HYSPARSE_GATHER_KERNEL=tc|mma overrides the default.
+bool use_gather_tc(const Shape &s) {
+    if (!sparse_gather_tc_supported(s)) return false;
+    const char *e = getenv("HYSPARSE_GATHER_KERNEL");
+    if (e && strcmp(e, "tc") == 0) return true;
+    return false;
+}
+
 // mask_ready: the dense path's selection bitmask in `ws` was already built
 // from this very index set (hysparse_block builds it once for all its layers).
 int run_sparse(const Shape &s, const void *q, const void *k, const void *v, const int32_t *idx,
@@ -167,6 +177,9 @@ int run_sparse(const Shape &s, const void *q, const void *k, const void *v, cons
         return cuda_status(sparse_dense_tc_launch(s, q, k, v, idx, topk, gate, window, out, og, ol, mask,
                                                   status, wait_limit_ns(), st));
     }
+    if (use_gather_tc(s))
+        return cuda_status(sparse_gather_tc_launch(s, q, k, v, idx, topk, gate, window, out, og, ol, status,
+                                                   wait_limit_ns(), st));
     if (sparse_mma_supported(s))
         return cuda_status(sparse_attn_mma_launch(s, q, k, v, idx, topk, gate, window, out, og, ol, status,
                                                   wait_limit_ns(), st));

@@ -56,6 +56,14 @@ cudaError_t sparse_attn_mma_launch(const Shape &s, const void *q, const void *k,
                                    void *og, void *ol, unsigned int *status, unsigned long long wait_ns,
                                    cudaStream_t st);
 
+// sparse_gather_tc.cu (bf16, d = 128, G <= 16, contiguous caches): the
+// sparse layer as a row gather on the tcgen05 tensor cores
+bool sparse_gather_tc_supported(const Shape &s);
+cudaError_t sparse_gather_tc_launch(const Shape &s, const void *q, const void *k, const void *v,
+                                    const int32_t *idx, int topk, const float *gate, int window, void *out,
+                                    void *og, void *ol, unsigned int *status, unsigned long long wait_ns,
+                                    cudaStream_t st);
+
 // sparse_mma.cu, decode full layer (bf16, d = 128, G <= 16, Lq == 1): split-K
 // partials + logit stash in `ws` (decode_ws_bytes of it), then a combine.
 size_t decode_ws_bytes(const Shape &s);

@@ -258,12 +258,16 @@ SWEEP = [
 
 @pytest.fixture
 def sparse_path(request, monkeypatch):
-    """Force one sparse-layer kernel (dense-masked tcgen05 or gather) for
-    the test; None keeps the library's own choice."""
-    if request.param is None:
-        monkeypatch.delenv("HYSPARSE_SPARSE_PATH", raising=False)
-    else:
-        monkeypatch.setenv("HYSPARSE_SPARSE_PATH", request.param)
+    """Force one sparse-layer kernel for the test: "dense" (dense-masked
+    tcgen05 tiles), "gather" (warp-MMA row gather) or "gather_tc" (tcgen05
+    row gather); None keeps the library's own choice."""
+    monkeypatch.delenv("HYSPARSE_SPARSE_PATH", raising=False)
+    monkeypatch.delenv("HYSPARSE_GATHER_KERNEL", raising=False)
+    if request.param == "dense":
+        monkeypatch.setenv("HYSPARSE_SPARSE_PATH", "dense")
+    elif request.param in ("gather", "gather_tc"):
+        monkeypatch.setenv("HYSPARSE_SPARSE_PATH", "gather")
+        monkeypatch.setenv("HYSPARSE_GATHER_KERNEL", "tc" if request.param == "gather_tc" else "mma")
     return request.param
 
 
@@ -271,8 +275,8 @@ def _sweep_params():
     out = []
     for c in SWEEP:
         paths = [None]
-        if c[7] == "bf16" and c[2] >= 64:
-            paths = ["gather", "dense"]
+        if c[7] == "bf16":
+            paths = ["gather", "gather_tc"] + (["dense"] if c[2] >= 64 else [])
         for pth in paths:
             out.append(pytest.param(c, pth, id=f"{c[0]}-{pth or 'auto'}"))
     return out
@@ -290,7 +294,7 @@ def test_shape_sweep_all_rows(case, sparse_path):
     oracle_check_rows(inp, w, rows, out, lse, idx, sc, outs)
 
 
-@pytest.mark.parametrize("sparse_path", ["dense", "gather"], indirect=True)
+@pytest.mark.parametrize("sparse_path", ["dense", "gather", "gather_tc"], indirect=True)
 def test_global_branch_far_below_unselected_keys(sparse_path):
     """Unselected keys whose logits sit ~200 (log2 units) above every selected
     key: a softmax reference taken over all keys would underflow every
@@ -329,7 +333,8 @@ def test_global_branch_far_below_unselected_keys(sparse_path):
 FULL = [pytest.param("prefill8k", "gather", id="prefill8k-gather"),
         pytest.param("prefill8k", "dense", id="prefill8k-dense"),
         pytest.param("prefill32k", None, id="prefill32k-auto"),
-        pytest.param("moe64k", None, id="moe64k-auto")]
+        pytest.param("moe64k", None, id="moe64k-auto"),
+        pytest.param("moe64k", "gather_tc", id="moe64k-gather_tc")]
 
 
 @pytest.mark.parametrize("name,sparse_path", FULL, indirect=["sparse_path"])
@@ -353,7 +358,8 @@ def test_full_size_prefill_sampled_rows(name, sparse_path):
     check_sparse_on_oracle_idx(inp, w, rows, idx, o_idx, tag=f"{name}: ")
 
 
-def test_full_size_decode_sampled_batches():
+@pytest.mark.parametrize("sparse_path", [None, "gather", "gather_tc"], indirect=True)
+def test_full_size_decode_sampled_batches(sparse_path):
     w = gen.WORKLOADS["decode"]
     inp = gen.make_inputs(w, seed=0, device=DEV)
     out, lse, idx, outs_list = hs.block(inp["q"], inp["k"], inp["v"], inp["q_sparse"], inp["gate"],
