@@ -21,12 +21,12 @@
 // head so that one head's K and V stay in L2):
 //   warps 0-3  softmax: thread t owns key slot t of a chunk (TMEM lane t of
 //              S^T) and, in the epilogue, output column d = t (lane t of O^T)
-//   warps 4-5  producers: gather the chunk's 128 K rows and 128 V rows with
-//              16-byte cp.async into 128-byte-swizzled K-major tiles (a key
-//              that is -1 or out of range is zero-filled), plus the item's
-//              query rows; a 3-slot ring of 32 KB tiles in MMA order
-//              K0, K1, V0, K2, V1, ...
-//   warp 6     MMA issuer (one thread)
+//   warp 4     producer: gathers the chunk's 128 K rows and 128 V rows with
+//              TMA tile::gather4 loads (four 128-byte row halves per
+//              instruction, 128-byte swizzled K-major as the MMA reads them),
+//              plus the item's query rows with a tiled TMA load; a 3-slot ring
+//              of 32 KB tiles in MMA order K0, K1, V0, K2, V1, ...
+//   warp 5     MMA issuer (one thread)
 // Per-head softmax statistics need a reduction over the keys, i.e. across
 // TMEM lanes: each warp takes its 16 maxima with redux.sync.max.f32, and the
 // warps agree through one barrier reduction whether any head's reference
@@ -41,6 +41,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc_attn.cuh"
 #include "tc_util.cuh"
 
 namespace hs {
@@ -57,8 +58,8 @@ constexpr int HALF_B = TILE_B / 2;   // one 64-column swizzled half
 constexpr int QP_B = NH * 256;       // Q or one P buffer: 16 rows x 128 bf16
 constexpr int QP_HALF = QP_B / 2;
 constexpr int SOFT_WARPS = 4, PROD_WARPS = 1, MMA_WARP = SOFT_WARPS + PROD_WARPS;
+constexpr int KPL = 4;               // keys of a chunk per producer lane (rows 4 l .. 4 l + 3)
 constexpr int THREADS = 32 * (MMA_WARP + 1);
-constexpr int PROD_THREADS = 32 * PROD_WARPS;
 constexpr uint32_t TMEM_COLS = 64;   // S0 | S1 | O_global | O_local, 16 columns each
 constexpr float kLazy = 8.0f;        // log2 units a chunk maximum may exceed the reference by
 constexpr uint64_t kDrainNs = 1000000000ull;
@@ -135,16 +136,26 @@ __device__ __forceinline__ Item item_of(const Params &p, long long it) {
 __device__ __forceinline__ int seq_k(int j) { return j == 0 ? 0 : 2 * j - 1; }
 __device__ __forceinline__ int seq_v(int j, int n) { return j + 1 < n ? 2 * j + 2 : 2 * j + 1; }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-                 : "memory");
+// TMA gather of four rows (tile::gather4, 2-D map, one-row box): the box's
+// columns of rows r0..r3 land as four consecutive box rows at dst.  Signals
+// `bar` with the bytes written.  No multicast.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *m, uint32_t bar, int x, int r0, int r1,
+                                            int r2, int r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
 }
-// Arrive on `bar` when every cp.async this thread has issued so far has
-// completed; the arrival counts toward the barrier's expected count.
-__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+
+// 2-D tiled TMA load; signals `bar` with the bytes written.  No multicast.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *m, uint32_t bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ float redux_max(float x) {
     float r;
@@ -207,35 +218,40 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// Key of list entry / window slot t of chunk j (-1: none or out of range).
-__device__ __forceinline__ int chunk_key(const Params &p, const int32_t *list, const Item &it, int j, int t,
-                                         bool report_bad) {
+// Raw key of list entry / window slot t of chunk j: the list entry as
+// stored (not yet checked), the window key, or -1 past the list or window.
+// Loads are issued well ahead of their use and checked by key_checked at use,
+// so that no warp stalls on an index load it does not need yet.
+__device__ __forceinline__ int chunk_key_raw(const Params &p, const int32_t *list, const Item &it, int j, int t) {
     if (j < it.n_g) {
         const int e = j * CK + t;
-        if (e >= p.topk) return -1;
-        int key = __ldg(list + e);
-        if (key < -1 || key > it.pos) {
-            if (report_bad) report(p.status, HS_ERR_INVALID_INDEX);
-            key = -1;
-        }
-        return key;
+        return e < p.topk ? __ldg(list + e) : -1;
     }
     const int key = it.lo + (j - it.n_g) * CK + t;
     return key <= it.pos ? key : -1;
+}
+
+// A raw key checked against the row's causal range: -1 for none; an entry
+// outside [-1, pos] is dropped (and reported when report_bad).
+__device__ __forceinline__ int key_checked(const Params &p, int key, int pos, bool report_bad) {
+    if (key < -1 || key > pos) {
+        if (report_bad) report(p.status, HS_ERR_INVALID_INDEX);
+        return -1;
+    }
+    return key;
 }
 
 __device__ __forceinline__ const int32_t *list_of(const Params &p, const Item &it) {
     return p.idx + (((size_t)it.b * p.Hkv + it.g) * p.Lq + it.i) * p.topk;
 }
 
-// Byte offset of 16-byte column chunk c16 (0..15) of row r in a K-major,
-// 128-byte-swizzled tile whose two 64-column halves are `half_bytes` apart.
-__device__ __forceinline__ uint32_t sw128(int r, int c16, uint32_t half_bytes) {
-    return (uint32_t)(c16 >> 3) * half_bytes + (uint32_t)r * 128u + ((uint32_t)((c16 & 7) ^ (r & 7)) << 4);
-}
+// Registers per thread: two CTAs of THREADS threads share the SM's 65536.
+template <int NS>
+constexpr int max_regs() { return Cfg<NS>::CTAS == 2 ? (65536 / (2 * THREADS)) / 8 * 8 : 255; }
 
 template <int NS>
-__global__ void __launch_bounds__(THREADS, Cfg<NS>::CTAS) sparse_gather_tc(const Params p) {
+__global__ void __launch_bounds__(THREADS) __maxnreg__(max_regs<NS>()) sparse_gather_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                 const __grid_constant__ CUtensorMap tv, const Params p) {
     constexpr size_t kRing = Cfg<NS>::kRing;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -247,7 +263,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<NS>::CTAS) sparse_gather_tc(const
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
-            mbar_init(smem_u32(&bars->kv_full[s]), PROD_THREADS);
+            mbar_init(smem_u32(&bars->kv_full[s]), 1);
             mbar_init(smem_u32(&bars->kv_empty[s]), 1);
         }
         mbar_init(smem_u32(&bars->q_empty), 1);
@@ -274,89 +290,96 @@ __global__ void __launch_bounds__(THREADS, Cfg<NS>::CTAS) sparse_gather_tc(const
 
     if (warp >= SOFT_WARPS && warp < MMA_WARP) {
         // ------------------------------------------------------ producer warp
-        const int half = lane >> 4, part = lane & 15;
+        // Lane l fetches rows 4l .. 4l+3 of every tile with TMA gathers: one
+        // tile::gather4 per 64-column half moves four whole 128-byte row halves,
+        // 128-byte swizzled as the MMA reads them, and the TMA unit signals the
+        // slot's full barrier with the bytes it wrote.
+        if (lane == 0) {
+            tma_prefetch(&tq);
+            tma_prefetch(&tk);
+            tma_prefetch(&tv);
+        }
         int seq = 0, item_n = 0;
         bool ok = true;
+        // look-ahead over the CTA's stream of chunks (items in order, their
+        // chunks in order): the keys of the chunk two K tiles ahead are loaded
+        // while the warp waits, across item boundaries too; they are checked
+        // against the row's range only at use
+        long long la_item = blockIdx.x;
+        Item la = item_of(p, la_item);
+        int la_j = 0;
+        auto la_keys = [&](int (&dst)[KPL]) {
+            const bool live = la_item < p.n_items;
+#pragma unroll
+            for (int u = 0; u < KPL; ++u)
+                dst[u] = live ? chunk_key_raw(p, list_of(p, la), la, la_j, 4 * lane + u) : -1;
+            if (live && ++la_j == la.n) {
+                la_j = 0;
+                la_item += stride;
+                if (la_item < p.n_items) la = item_of(p, la_item);
+            }
+        };
+        int ka[KPL], kp[KPL], kn[KPL], knn[KPL];
+#pragma unroll
+        for (int u = 0; u < KPL; ++u) ka[u] = kp[u] = -1;
+        la_keys(kn);
+        la_keys(knn);
         for (long long it_ = blockIdx.x; ok && it_ < p.n_items; it_ += stride, ++item_n) {
             const Item it = item_of(p, it_);
-            const int32_t *list = list_of(p, it);
-            const __nv_bfloat16 *kb = p.k + ((size_t)it.b * p.Lkv * p.Hkv + it.g) * 128;
-            const __nv_bfloat16 *vb = p.v + ((size_t)it.b * p.Lkv * p.Hkv + it.g) * 128;
-            const size_t qrow = ((size_t)it.b * p.Lq + it.i) * p.Hq + (size_t)it.g * p.G;
-            // keys of this lane's four rows (lane + 32 u): ka of the latest K chunk
-            // jk, kp of chunk jk - 1, kn of chunk jk + 1 (loaded one K tile ahead,
-            // while the warp waits for a free slot)
-            int jk = -1, ka[4], kp[4], kn[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                ka[u] = kp[u] = -1;
-                kn[u] = chunk_key(p, list, it, 0, 32 * u + lane, true);
-            }
+            const int row0 = it.b * p.Lkv;                    // key 0 of this sequence in the [B*Lkv] rows
+            const int col0 = it.g * 128;                      // this KV head's columns
+            const int qr = (it.b * p.Lq + it.i) * p.Hq + it.g * p.G;   // first query row of the group
+            int jk = -1;
             for (int t = 0; t < 2 * it.n; ++t) {
                 // production order: K0, then (K_{j+1}, V_j) pairs, then the last V
                 int j, is_v;
                 if (t == 0) { j = 0; is_v = 0; }
                 else if (t == 2 * it.n - 1) { j = it.n - 1; is_v = 1; }
                 else { is_v = (t & 1) == 0; j = is_v ? (t - 2) / 2 : (t + 1) / 2; }
-                int key[4];
+                int key[KPL];
                 if (!is_v) {
                     jk = j;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < KPL; ++u) {
                         kp[u] = ka[u];
-                        ka[u] = kn[u];
+                        ka[u] = key_checked(p, kn[u], it.pos, true);   // loaded two K tiles ago
+                        kn[u] = knn[u];
                         key[u] = ka[u];
                     }
-                    if (j + 1 < it.n) {
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) kn[u] = chunk_key(p, list, it, j + 1, 32 * u + lane, true);
-                    }
+                    la_keys(knn);
                 } else {                   // the item's last V follows its own K; else V_{jk-1}
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) key[u] = j == jk ? ka[u] : kp[u];
+                    for (int u = 0; u < KPL; ++u) key[u] = j == jk ? ka[u] : kp[u];
                 }
                 const int slot = seq % NS, use = seq / NS;
-                // every lane takes part in the shuffles below: the warp agrees on the wait
                 if (!(ok = __all_sync(0xffffffffu, wait_sleep(smem_u32(&bars->kv_empty[slot]), (use & 1) ^ 1,
                                                               p.wait_ns, abort))))
                     break;
-                const uint32_t tb = smem_u32(ring + slot * TILE_B);
-                if (t == 0) {
-                    // the item's query rows travel in the same copy group as K0: the
-                    // previous item's last S = K Q^T must have finished reading Q
-                    if (!(ok = __all_sync(0xffffffffu, wait_sleep(smem_u32(&bars->q_empty), (item_n & 1) ^ 1,
-                                                                  p.wait_ns, abort))))
-                        break;
+                if (t == 0 && !(ok = __all_sync(0xffffffffu, wait_sleep(smem_u32(&bars->q_empty), (item_n & 1) ^ 1,
+                                                                        p.wait_ns, abort))))
+                    break;   // the previous item's last S = K Q^T must have read Q
+                const uint32_t fb = smem_u32(&bars->kv_full[slot]);
+                if (lane == 0) mbar_expect_tx(fb, TILE_B + (t == 0 ? QP_B : 0));
+                __syncwarp();
+                if (t == 0 && lane < 2)   // the group's query rows (rows past the tensor read as zeros)
+                    tma_load_2d(smem_u32(sq) + lane * QP_HALF, &tq, fb, lane * 64, qr);
+                // a key that is -1 (or was dropped) fetches key 0's row, which the
+                // softmax masks out: every row written is finite data
+                int r[KPL];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int e = lane * 8 + u;            // 0..255: head e/16, chunk e%16
-                        const int h = e >> 4, c16 = e & 15;
-                        const bool val = h < p.G;
-                        cp_async16(smem_u32(sq) + sw128(h, c16, QP_HALF),
-                                   p.q + (val ? (qrow + h) * 128 + c16 * 8 : 0), val);
-                    }
-                }
-                const __nv_bfloat16 *src = (is_v ? vb : kb) + part * 8;
-                const uint32_t dbase = tb + (uint32_t)(part >> 3) * HALF_B;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-#pragma unroll
-                    for (int r2 = 0; r2 < 16; ++r2) {
-                        // two rows per instruction: lanes 0-15 row 32 u + 2 r2, lanes 16-31 the next
-                        const int rl = 2 * r2 + half, row = 32 * u + rl;
-                        const int kr = __shfl_sync(0xffffffffu, key[u], rl);
-                        const bool val = kr >= 0;
-                        cp_async16(dbase + (uint32_t)row * 128u + ((uint32_t)((part & 7) ^ (row & 7)) << 4),
-                                   src + (val ? (size_t)kr * p.Hkv * 128 : 0), val);
-                    }
-                }
-                // the slot's full barrier counts this thread's arrival once all its
-                // copies so far have landed
-                cp_async_arrive_noinc(smem_u32(&bars->kv_full[slot]));
+                for (int u = 0; u < KPL; ++u) r[u] = row0 + (key[u] >= 0 ? key[u] : 0);
+                const CUtensorMap *m = is_v ? &tv : &tk;
+                const uint32_t tb = smem_u32(ring + slot * TILE_B) + (uint32_t)lane * 4u * 128u;
+                tma_gather4(tb, m, fb, col0, r[0], r[1], r[2], r[3]);
+                tma_gather4(tb + HALF_B, m, fb, col0 + 64, r[0], r[1], r[2], r[3]);
                 ++seq;
             }
         }
-        cp_async_wait_all();   // no copy of ours is still in flight when the CTA exits
+        if (lane == 0 && *abort) {
+            // let our own copies land before the CTA goes away
+            for (int s2 = seq > NS ? seq - NS : 0; s2 < seq; ++s2)
+                mbar_drain(smem_u32(&bars->kv_full[s2 % NS]), (s2 / NS) & 1);
+        }
     } else if (warp == MMA_WARP) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -370,7 +393,6 @@ __global__ void __launch_bounds__(THREADS, Cfg<NS>::CTAS) sparse_gather_tc(const
                 auto issue_s = [&](int j) -> bool {
                     const int c = gc + j, tk = T + seq_k(j), slot = tk % NS;
                     if (!wait_sleep(smem_u32(&bars->kv_full[slot]), (tk / NS) & 1, p.wait_ns, abort)) return false;
-                    fence_proxy_async_smem();   // copies landed through the generic proxy; the MMA reads async
                     if (!wait_sleep(smem_u32(&bars->s_free[c & 1]), ((c >> 1) & 1) ^ 1, p.wait_ns, abort))
                         return false;
                     tc_fence_after();
@@ -390,9 +412,8 @@ __global__ void __launch_bounds__(THREADS, Cfg<NS>::CTAS) sparse_gather_tc(const
                 if (!(ok = issue_s(0))) break;
                 for (int j = 0; j < it.n; ++j) {
                     if (j + 1 < it.n && !(ok = issue_s(j + 1))) break;
-                    const int c = gc + j, tv = T + seq_v(j, it.n), slot = tv % NS;
-                    if (!(ok = wait_sleep(smem_u32(&bars->kv_full[slot]), (tv / NS) & 1, p.wait_ns, abort))) break;
-                    fence_proxy_async_smem();
+                    const int c = gc + j, tv_ = T + seq_v(j, it.n), slot = tv_ % NS;
+                    if (!(ok = wait_sleep(smem_u32(&bars->kv_full[slot]), (tv_ / NS) & 1, p.wait_ns, abort))) break;
                     if (!(ok = wait_sleep(smem_u32(&bars->p_full[c & 1]), (c >> 1) & 1, p.wait_ns, abort))) break;
                     tc_fence_after();
                     const uint32_t va = smem_u32(ring + slot * TILE_B);
@@ -429,7 +450,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<NS>::CTAS) sparse_gather_tc(const
             float m[NH], lp_g[NH], lp_l[NH];
 #pragma unroll
             for (int h = 0; h < NH; ++h) { m[h] = -INFINITY; lp_g[h] = 0.f; lp_l[h] = 0.f; }
-            int key_next = chunk_key(p, list, it, 0, t, false);
+            int key_next = chunk_key_raw(p, list, it, 0, t);
             for (int j = 0; j < it.n; ++j) {
                 const int c = gc + j;
                 if (wg_any(bad || *abort)) break;
@@ -439,8 +460,8 @@ __global__ void __launch_bounds__(THREADS, Cfg<NS>::CTAS) sparse_gather_tc(const
 #pragma unroll
                     for (int h = 0; h < NH; ++h) m[h] = -INFINITY;   // the window branch starts afresh
                 }
-                const bool valid = key_next >= 0;
-                if (j + 1 < it.n) key_next = chunk_key(p, list, it, j + 1, t, false);
+                const bool valid = key_checked(p, key_next, it.pos, false) >= 0;
+                if (j + 1 < it.n) key_next = chunk_key_raw(p, list, it, j + 1, t);
                 bad |= !__all_sync(0xffffffffu, wait_sleep(smem_u32(&bars->s_full[c & 1]), (c >> 1) & 1,
                                                           p.wait_ns, abort));
                 tc_fence_after();
@@ -622,8 +643,30 @@ bool sparse_gather_tc_supported(const Shape &s) {
 }
 
 namespace {
+// 2-D map over a bf16 matrix of `rows` rows of `cols` elements (row pitch
+// `cols` elements), a {64, box_rows} box, 128-byte swizzle; rows past the end
+// read as zeros.
+bool make_map_2d(CUtensorMap *m, const void *base, long long cols, long long rows, int box_rows) {
+    auto enc = tc::encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int NS>
 cudaError_t launch_ns(const gtc::Params &p0, cudaStream_t st) {
+    CUtensorMap mq, mk, mv;
+    // K and V as [B*Lkv rows][Hkv*128] (one gathered row = one key's KV-head slice,
+    // one-row box for tile::gather4); Q as [B*Lq*Hq rows][128] with a 16-row box
+    if (!make_map_2d(&mk, p0.k, (long long)p0.Hkv * 128, (long long)p0.B * p0.Lkv, 1) ||
+        !make_map_2d(&mv, p0.v, (long long)p0.Hkv * 128, (long long)p0.B * p0.Lkv, 1) ||
+        !make_map_2d(&mq, p0.q, 128, (long long)p0.B * p0.Lq * p0.Hq, gtc::NH))
+        return cudaErrorInvalidValue;
     using namespace gtc;
     static bool attr = false;
     if (!attr) {
@@ -639,7 +682,7 @@ cudaError_t launch_ns(const gtc::Params &p0, cudaStream_t st) {
     const long long slots = (long long)Cfg<NS>::CTAS * sms;
     const long long per = (p0.n_items + slots - 1) / slots;
     const long long grid = (p0.n_items + per - 1) / per;
-    sparse_gather_tc<NS><<<(unsigned)grid, THREADS, Cfg<NS>::kSmem, st>>>(p0);
+    sparse_gather_tc<NS><<<(unsigned)grid, THREADS, Cfg<NS>::kSmem, st>>>(mq, mk, mv, p0);
     count_launch();
     return cudaGetLastError();
 }

@@ -106,21 +106,26 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Gather the K and V rows of list entries [t0, t0+32) into `stage` and commit
-// them as one cp.async group.  Lane l validates entry t0+l; the 32 rows are
-// then copied two per instruction (16 lanes x 16 bytes per 256-byte row).
-__device__ __forceinline__ void issue_chunk(const SpParams &p, const int32_t *list, bool from_list, int lo,
-                                            int n_list, int t0, int pos, const __nv_bfloat16 *kb,
+// Lane l's entry of chunk c (entry c*32 + l) as stored: the list entry, the
+// window key, or -1 past the list.  Loaded one chunk before the chunk is
+// issued, so that no warp waits on an index load it is about to use.
+__device__ __forceinline__ int chunk_entry(const int32_t *list, bool from_list, int lo, int n_list, int c, int lane) {
+    const int t = c * CH + lane;
+    if (t >= n_list) return -1;
+    return from_list ? __ldg(list + t) : lo + t;
+}
+
+// Gather the K and V rows of one chunk's 32 entries into `stage` and commit
+// them as one cp.async group.  Lane l holds entry l (`entry`, as stored) and
+// validates it here; the 32 rows are then copied two per instruction (16
+// lanes x 16 bytes per 256-byte row).
+__device__ __forceinline__ void issue_chunk(const SpParams &p, int entry, int pos, const __nv_bfloat16 *kb,
                                             const __nv_bfloat16 *vb, uint8_t *stage, uint32_t &vmask, int lane,
                                             const int32_t *table) {
-    const int t = t0 + lane;
-    int key = -1;
-    if (t < n_list) {
-        key = from_list ? __ldg(list + t) : lo + t;
-        if (key < -1 || key > pos) {
-            report(p.status, HS_ERR_INVALID_INDEX);
-            key = -1;
-        }
+    int key = entry;
+    if (key < -1 || key > pos) {
+        report(p.status, HS_ERR_INVALID_INDEX);
+        key = -1;
     }
     // row of the key in the cache (kb, vb): the key itself, or its row in the
     // page pool when the cache is paged (a page outside the pool is reported
@@ -283,12 +288,13 @@ __device__ __forceinline__ void run_branch(const WarpCtx &w, bool from_list, con
     const int n_list = from_list ? p.topk : w.pos - w.lo + 1;
     const int nch = (n_list + CH - 1) / CH;
     uint32_t vm0 = 0, vm1 = 0, vm2 = 0;
+    int entry = chunk_entry(w.list, from_list, w.lo, n_list, 0, w.lane);   // of the next chunk to issue
     auto issue = [&](int c) {
         const int s = c % ST;
         uint32_t vmask = 0;
         if (c < nch) {
-            issue_chunk(p, w.list, from_list, w.lo, n_list, c * CH, w.pos, w.kb, w.vb, w.wbase + s * STAGE_BYTES,
-                        vmask, w.lane, w.table);
+            issue_chunk(p, entry, w.pos, w.kb, w.vb, w.wbase + s * STAGE_BYTES, vmask, w.lane, w.table);
+            entry = chunk_entry(w.list, from_list, w.lo, n_list, c + 1, w.lane);
         } else {
             cp_async_commit();
         }
