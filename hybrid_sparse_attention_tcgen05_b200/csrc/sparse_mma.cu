@@ -19,6 +19,8 @@
 // same pipeline over the contiguous key range; both branches are merged by
 // the gate in registers and the G output rows are written once.
 #include <cuda_bf16.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -28,22 +30,34 @@ namespace hs {
 namespace tc {
 namespace {
 
-constexpr int CH = 32;            // keys per chunk (one per lane)
-constexpr int RS = 272;           // padded row stride in shared memory (bytes)
-constexpr int STAGE_BYTES = 2 * CH * RS;
+constexpr int RS = 256;
+// Stages of the 8-head configuration (3 with 4 warps, or 2 with 7 warps).
+constexpr int mma_stages_g8() { return 2; }           // row stride in shared memory (bytes): one K or V row
 
-// Per head-block count NB (heads padded to 8*NB): SW warps (items) per CTA,
-// each with an ST-stage chunk ring and its Q staging.  Groups of up to 8
-// heads keep three stages (4 warps); 16-head groups trade a stage for a
-// fifth warp on the SM (measured: 3 % faster at the 64k, 16-head workload,
-// 5 % slower for 4-head decode).
-template <int NB>
+// Byte offset of 16-byte chunk c16 (0..15) of row r of a staged tile: the
+// chunks of a row are XOR-permuted by r mod 8, so the eight rows an ldmatrix
+// reads at one column fall in eight different bank groups (conflict-free at a
+// 256-byte stride, without padding).
+__device__ __forceinline__ uint32_t sw_off(int r, int c16) {
+    return (uint32_t)r * RS + ((uint32_t)(c16 ^ (r & 7)) << 4);
+}
+
+// Per head-block count NB (heads padded to 8*NB) and keys per chunk CK (16
+// or 32): SW warps (items) per CTA, each with an ST-stage chunk ring.  A
+// warp stages its query rows (and, at the end, its output rows) in the ring's
+// last stage, which the pipeline only fills after the rows are in registers.
+// Measured at the 64k-token, 16-head workload: 32-key chunks, two stages,
+// and as many warps as shared memory holds (each warp is an independent
+// gather stream; more of them keep more bytes in flight).
+template <int NB, int CK>
 struct SpSmem {
-    static constexpr int SW = NB == 1 ? 4 : 5;
-    static constexpr int ST = NB == 1 ? 3 : 2;
-    static constexpr int QB = 8 * NB * RS;               // Q staging / output staging
-    static constexpr int WARP_BYTES = ST * STAGE_BYTES + QB;
+    static constexpr int ST = NB == 1 ? mma_stages_g8() : (CK == 16 ? 4 : 2);
+    static constexpr int SW = NB == 1 ? (ST == 3 ? 4 : 7) : (CK == 16 ? 6 : 7);
+    static constexpr int STAGE_BYTES = 2 * CK * RS;
+    static constexpr int WARP_BYTES = ST * STAGE_BYTES;
     static constexpr size_t bytes = (size_t)SW * WARP_BYTES;
+    static_assert(8 * NB * RS <= STAGE_BYTES, "query / output staging fits one stage");
+    static_assert(bytes <= 232448, "shared memory per CTA");
 };
 
 __device__ __forceinline__ float ex2f(float x) {
@@ -109,9 +123,10 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // Lane l's entry of chunk c (entry c*32 + l) as stored: the list entry, the
 // window key, or -1 past the list.  Loaded one chunk before the chunk is
 // issued, so that no warp waits on an index load it is about to use.
+template <int CK>
 __device__ __forceinline__ int chunk_entry(const int32_t *list, bool from_list, int lo, int n_list, int c, int lane) {
-    const int t = c * CH + lane;
-    if (t >= n_list) return -1;
+    const int t = c * CK + lane;
+    if (lane >= CK || t >= n_list) return -1;
     return from_list ? __ldg(list + t) : lo + t;
 }
 
@@ -119,6 +134,7 @@ __device__ __forceinline__ int chunk_entry(const int32_t *list, bool from_list, 
 // them as one cp.async group.  Lane l holds entry l (`entry`, as stored) and
 // validates it here; the 32 rows are then copied two per instruction (16
 // lanes x 16 bytes per 256-byte row).
+template <int CK>
 __device__ __forceinline__ void issue_chunk(const SpParams &p, int entry, int pos, const __nv_bfloat16 *kb,
                                             const __nv_bfloat16 *vb, uint8_t *stage, uint32_t &vmask, int lane,
                                             const int32_t *table) {
@@ -143,59 +159,60 @@ __device__ __forceinline__ void issue_chunk(const SpParams &p, int entry, int po
     const uint32_t sbase = smem_u32(stage);
     const int half = lane >> 4, part = lane & 15;
 #pragma unroll
-    for (int r2 = 0; r2 < CH / 2; ++r2) {
+    for (int r2 = 0; r2 < CK / 2; ++r2) {
         const int row = 2 * r2 + half;
         const int kr = __shfl_sync(0xffffffffu, key, row);
         const bool ok = kr >= 0;
         const size_t so = ok ? (size_t)kr * p.Hkv * 128 + part * 8 : 0;
-        const uint32_t d = sbase + row * RS + part * 16;
+        const uint32_t d = sbase + sw_off(row, part);
         cp_async16(d, kb + so, ok);
-        cp_async16(d + CH * RS, vb + so, ok);
+        cp_async16(d + CK * RS, vb + so, ok);
     }
     cp_async_commit();
 }
 
-template <int NB>
+template <int NB, int CK>
 __device__ __forceinline__ void compute_chunk(const uint8_t *stage, uint32_t vmask, const uint32_t (&bq)[NB][8][2],
                                               float c2, Branch<NB> &br, int lane, float *stash = nullptr,
                                               long long stash_ld = 0, int j0 = 0, int G = 0, int j_lim = 0) {
     const uint32_t ks_base = smem_u32(stage);
-    const uint32_t vs_base = smem_u32(stage + CH * RS);
-    float c[NB][2][4];
+    constexpr int MT = CK / 16;   // 16-key MMA tiles per chunk
+    const uint32_t vs_base = smem_u32(stage + CK * RS);
+    float c[NB][MT][4];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
             for (int r = 0; r < 4; ++r) c[nb][mt][r] = 0.f;
-    // S^T[32 keys x 8NB heads] = K Q^T
+    // S^T[CK keys x 8NB heads] = K Q^T
     const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;
     const int acol = (lane >> 4) * 8;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
+        for (int mt = 0; mt < MT; ++mt) {
             uint32_t a0, a1, a2, a3;
-            ldsm_x4(ks_base + (16 * mt + arow) * RS + (16 * ks + acol) * 2, a0, a1, a2, a3);
+            ldsm_x4(ks_base + sw_off(16 * mt + arow, 2 * ks + (acol >> 3)), a0, a1, a2, a3);
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) mma16816(c[nb][mt], a0, a1, a2, a3, bq[nb][ks][0], bq[nb][ks][1]);
         }
     }
     // online softmax per head column (keys spread over lane/4 and the two row halves)
-    bool kv[2][2];
+    bool kv[MT][2];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int rh = 0; rh < 2; ++rh) kv[mt][rh] = (vmask >> (16 * mt + (lane >> 2) + 8 * rh)) & 1u;
-    uint32_t bp[NB][2][2];
+    uint32_t bp[NB][MT][2];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            float x[2][2];
+            float x[MT][2];
             float cm = -INFINITY;
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
+            for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
                 for (int rh = 0; rh < 2; ++rh) {
                     x[mt][rh] = kv[mt][rh] ? c[nb][mt][2 * rh + e] * c2 : -INFINITY;
@@ -216,7 +233,7 @@ __device__ __forceinline__ void compute_chunk(const uint8_t *stage, uint32_t vma
             const float corr = (mn == -INFINITY) ? 1.f : ex2f(br.m[nb][e] - mn);
             float ps = 0.f;
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
+            for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
                 for (int rh = 0; rh < 2; ++rh) {
                     const float pv = (mn == -INFINITY) ? 0.f : ex2f(x[mt][rh] - mn);
@@ -236,7 +253,7 @@ __device__ __forceinline__ void compute_chunk(const uint8_t *stage, uint32_t vma
         }
         // P^T fragments (keys x heads) -> B operand (k = keys, n = heads)
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
+        for (int mt = 0; mt < MT; ++mt) {
             bp[nb][mt][0] = movm_t(pack_bf16(c[nb][mt][0], c[nb][mt][1]));
             bp[nb][mt][1] = movm_t(pack_bf16(c[nb][mt][2], c[nb][mt][3]));
         }
@@ -247,9 +264,9 @@ __device__ __forceinline__ void compute_chunk(const uint8_t *stage, uint32_t vma
 #pragma unroll
     for (int md = 0; md < 8; ++md) {
 #pragma unroll
-        for (int kt = 0; kt < 2; ++kt) {
+        for (int kt = 0; kt < MT; ++kt) {
             uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(vs_base + (16 * kt + vrow) * RS + (16 * md + vcol) * 2, a0, a1, a2, a3);
+            ldsm_x4_t(vs_base + sw_off(16 * kt + vrow, 2 * md + (vcol >> 3)), a0, a1, a2, a3);
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) mma16816(br.o[nb][md], a0, a1, a2, a3, bp[nb][kt][0], bp[nb][kt][1]);
         }
@@ -270,35 +287,36 @@ struct WarpCtx {
     int G = 0;
 };
 
-__device__ __forceinline__ uint32_t pick3(int s, uint32_t a, uint32_t b, uint32_t c) {
-    return s == 0 ? a : (s == 1 ? b : c);
+__device__ __forceinline__ uint32_t pick4(int s, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return s == 0 ? a : (s == 1 ? b : (s == 2 ? c : d));
 }
 
 // Run one branch (from_list: the top-k list, else the causal window) through
 // the ST-stage cp.async pipeline.  One group is committed per iteration (an
 // empty one past the end), so waiting for "at most ST-1 pending" always means
 // the chunk about to be used has landed.
-template <int NB>
+template <int NB, int CK>
 __device__ __forceinline__ void run_branch(const WarpCtx &w, bool from_list, const uint32_t (&bq)[NB][8][2],
                                            Branch<NB> &br) {
-    constexpr int ST = SpSmem<NB>::ST;
-    static_assert(ST == 2 || ST == 3, "pick3 holds two or three stages");
+    constexpr int ST = SpSmem<NB, CK>::ST;
+    constexpr int STAGE_BYTES = SpSmem<NB, CK>::STAGE_BYTES;
+    static_assert(ST >= 2 && ST <= 4, "pick4 holds two to four stages");
     const SpParams &p = *w.p;
     br.init();
     const int n_list = from_list ? p.topk : w.pos - w.lo + 1;
-    const int nch = (n_list + CH - 1) / CH;
-    uint32_t vm0 = 0, vm1 = 0, vm2 = 0;
-    int entry = chunk_entry(w.list, from_list, w.lo, n_list, 0, w.lane);   // of the next chunk to issue
+    const int nch = (n_list + CK - 1) / CK;
+    uint32_t vm0 = 0, vm1 = 0, vm2 = 0, vm3 = 0;
+    int entry = chunk_entry<CK>(w.list, from_list, w.lo, n_list, 0, w.lane);   // of the next chunk to issue
     auto issue = [&](int c) {
         const int s = c % ST;
         uint32_t vmask = 0;
         if (c < nch) {
-            issue_chunk(p, entry, w.pos, w.kb, w.vb, w.wbase + s * STAGE_BYTES, vmask, w.lane, w.table);
-            entry = chunk_entry(w.list, from_list, w.lo, n_list, c + 1, w.lane);
+            issue_chunk<CK>(p, entry, w.pos, w.kb, w.vb, w.wbase + s * STAGE_BYTES, vmask, w.lane, w.table);
+            entry = chunk_entry<CK>(w.list, from_list, w.lo, n_list, c + 1, w.lane);
         } else {
             cp_async_commit();
         }
-        if (s == 0) vm0 = vmask; else if (s == 1) vm1 = vmask; else vm2 = vmask;
+        if (s == 0) vm0 = vmask; else if (s == 1) vm1 = vmask; else if (s == 2) vm2 = vmask; else vm3 = vmask;
     };
     for (int c = 0; c < ST - 1; ++c) issue(c);
 #pragma unroll 1
@@ -308,18 +326,18 @@ __device__ __forceinline__ void run_branch(const WarpCtx &w, bool from_list, con
         cp_async_wait<ST - 1>();
         __syncwarp();
         const int s = c % ST;
-        compute_chunk<NB>(w.wbase + s * STAGE_BYTES, pick3(s, vm0, vm1, vm2), bq, w.c2, br, w.lane, w.stash,
-                          w.stash_ld, w.lo + c * CH, w.G, n_list - c * CH);
+        compute_chunk<NB, CK>(w.wbase + s * STAGE_BYTES, pick4(s, vm0, vm1, vm2, vm3), bq, w.c2, br, w.lane,
+                              w.stash, w.stash_ld, w.lo + c * CK, w.G, n_list - c * CK);
     }
     cp_async_wait<0>();
     __syncwarp();
 }
 
-template <int NB>
-__global__ void __launch_bounds__(SpSmem<NB>::SW * 32, 1) sparse_attn_mma(const SpParams p) {
+template <int NB, int CK>
+__global__ void __launch_bounds__(SpSmem<NB, CK>::SW * 32, 1) sparse_attn_mma(const SpParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long item = (long long)blockIdx.x * SpSmem<NB>::SW + warp;
+    const long long item = (long long)blockIdx.x * SpSmem<NB, CK>::SW + warp;
     if (item >= (long long)p.B * p.Lq * p.Hkv) return;   // whole warp leaves together
     // KV head slowest, then batch, then row: neighbouring warps gather from
     // the same KV head's cache (which stays in L2) and have similar row lengths
@@ -329,15 +347,16 @@ __global__ void __launch_bounds__(SpSmem<NB>::SW * 32, 1) sparse_attn_mma(const 
     const int g = (int)(head_batch / p.B);
     const int G = p.G;
     const int pos = seq_len(p, b) - p.Lq + i;
-    uint8_t *wbase = smem + warp * SpSmem<NB>::WARP_BYTES;
-    uint8_t *qs = wbase + SpSmem<NB>::ST * STAGE_BYTES;
+    uint8_t *wbase = smem + warp * SpSmem<NB, CK>::WARP_BYTES;
+    // query rows (and at the end the output rows) staged in the ring's last stage
+    uint8_t *qs = wbase + (SpSmem<NB, CK>::ST - 1) * SpSmem<NB, CK>::STAGE_BYTES;
     // stage the group's query rows (zero rows pad the heads up to 8*NB)
     const size_t qrow = ((size_t)b * p.Lq + i) * p.Hq + (size_t)g * G;
     for (int e = lane; e < 8 * NB * 16; e += 32) {
         const int h = e >> 4, cc = e & 15;
         uint4 val = make_uint4(0, 0, 0, 0);
         if (h < G) val = __ldg(reinterpret_cast<const uint4 *>(p.q + (qrow + h) * 128) + cc);
-        *reinterpret_cast<uint4 *>(qs + h * RS + cc * 16) = val;
+        *reinterpret_cast<uint4 *>(qs + sw_off(h, cc)) = val;
     }
     __syncwarp();
     uint32_t bq[NB][8][2];
@@ -345,7 +364,7 @@ __global__ void __launch_bounds__(SpSmem<NB>::SW * 32, 1) sparse_attn_mma(const 
     for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
         for (int kp = 0; kp < 4; ++kp)
-            ldsm_x4(smem_u32(qs + (8 * nb + (lane & 7)) * RS + (32 * kp + 8 * (lane >> 3)) * 2),
+            ldsm_x4(smem_u32(qs + sw_off(8 * nb + (lane & 7), 4 * kp + (lane >> 3))),
                     bq[nb][2 * kp][0], bq[nb][2 * kp][1], bq[nb][2 * kp + 1][0], bq[nb][2 * kp + 1][1]);
 
     WarpCtx w;
@@ -365,8 +384,8 @@ __global__ void __launch_bounds__(SpSmem<NB>::SW * 32, 1) sparse_attn_mma(const 
     w.lane = lane;
     w.c2 = p.scale_log2;
     Branch<NB> bg, bl;
-    run_branch<NB>(w, true, bq, bg);
-    run_branch<NB>(w, false, bq, bl);
+    run_branch<NB, CK>(w, true, bq, bg);
+    run_branch<NB, CK>(w, false, bq, bl);
 
     // gate merge, stage the G output rows in shared memory, write them once
     __syncwarp();
@@ -396,7 +415,8 @@ __global__ void __launch_bounds__(SpSmem<NB>::SW * 32, 1) sparse_attn_mma(const 
                     for (int rh = 0; rh < 2; ++rh) {
                         const int d = 16 * md + (lane >> 2) + 8 * rh;
                         const float val = bg.o[nb][md][2 * rh + e] * wg + bl.o[nb][md][2 * rh + e] * wl;
-                        reinterpret_cast<__nv_bfloat16 *>(qs + h * RS)[d] = __float2bfloat16_rn(val);
+                        *reinterpret_cast<__nv_bfloat16 *>(qs + sw_off(h, d >> 3) + (d & 7) * 2) =
+                            __float2bfloat16_rn(val);
                     }
             }
         }
@@ -404,7 +424,7 @@ __global__ void __launch_bounds__(SpSmem<NB>::SW * 32, 1) sparse_attn_mma(const 
         for (int e = lane; e < G * 16; e += 32) {
             const int h = e >> 4, cc = e & 15;
             reinterpret_cast<uint4 *>(dst + orow + (size_t)h * 128)[cc] =
-                *reinterpret_cast<const uint4 *>(qs + h * RS + cc * 16);
+                *reinterpret_cast<const uint4 *>(qs + sw_off(h, cc));
         }
         __syncwarp();
     }
@@ -430,12 +450,12 @@ struct DecParams {
     int nchunk;
 };
 
-template <int NB>
-__global__ void __launch_bounds__(SpSmem<NB>::SW * 32, 1) decode_full_mma(const DecParams dp) {
+template <int NB, int CK>
+__global__ void __launch_bounds__(SpSmem<NB, CK>::SW * 32, 1) decode_full_mma(const DecParams dp) {
     extern __shared__ __align__(128) uint8_t smem[];
     const SpParams &p = dp.sp;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long item = (long long)blockIdx.x * SpSmem<NB>::SW + warp;
+    const long long item = (long long)blockIdx.x * SpSmem<NB, CK>::SW + warp;
     if (item >= (long long)p.B * p.Hkv * dp.nchunk) return;
     // KV head fastest: neighbouring warps read the same keys' adjacent
     // 256-byte head slices of each 2 KB K and V row
@@ -444,14 +464,15 @@ __global__ void __launch_bounds__(SpSmem<NB>::SW * 32, 1) decode_full_mma(const 
     const int ch = (int)(rest % dp.nchunk);
     const int b = (int)(rest / dp.nchunk);
     const int G = p.G;
-    uint8_t *wbase = smem + warp * SpSmem<NB>::WARP_BYTES;
-    uint8_t *qs = wbase + SpSmem<NB>::ST * STAGE_BYTES;
+    uint8_t *wbase = smem + warp * SpSmem<NB, CK>::WARP_BYTES;
+    // query rows (and at the end the output rows) staged in the ring's last stage
+    uint8_t *qs = wbase + (SpSmem<NB, CK>::ST - 1) * SpSmem<NB, CK>::STAGE_BYTES;
     const size_t qrow = (size_t)b * p.Hq + (size_t)g * G;      // Lq == 1
     for (int e = lane; e < 8 * NB * 16; e += 32) {
         const int h = e >> 4, cc = e & 15;
         uint4 val = make_uint4(0, 0, 0, 0);
         if (h < G) val = __ldg(reinterpret_cast<const uint4 *>(p.q + (qrow + h) * 128) + cc);
-        *reinterpret_cast<uint4 *>(qs + h * RS + cc * 16) = val;
+        *reinterpret_cast<uint4 *>(qs + sw_off(h, cc)) = val;
     }
     __syncwarp();
     uint32_t bq[NB][8][2];
@@ -459,7 +480,7 @@ __global__ void __launch_bounds__(SpSmem<NB>::SW * 32, 1) decode_full_mma(const 
     for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
         for (int kp = 0; kp < 4; ++kp)
-            ldsm_x4(smem_u32(qs + (8 * nb + (lane & 7)) * RS + (32 * kp + 8 * (lane >> 3)) * 2),
+            ldsm_x4(smem_u32(qs + sw_off(8 * nb + (lane & 7), 4 * kp + (lane >> 3))),
                     bq[nb][2 * kp][0], bq[nb][2 * kp][1], bq[nb][2 * kp + 1][0], bq[nb][2 * kp + 1][1]);
     const int Lb = seq_len(p, b);
     const int lo = ch * kDecChunk;
@@ -484,7 +505,7 @@ __global__ void __launch_bounds__(SpSmem<NB>::SW * 32, 1) decode_full_mma(const 
     w.stash_ld = p.Lkv;
     w.G = G;
     Branch<NB> br;
-    if (lo < hi) run_branch<NB>(w, false, bq, br);
+    if (lo < hi) run_branch<NB, CK>(w, false, bq, br);
     else br.init();   // a chunk past this sequence's cache: an empty partial (m = -inf, l = 0, O = 0)
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)
@@ -543,39 +564,49 @@ __global__ void __launch_bounds__(256) decode_combine(const DecParams dp, float 
     }
 }
 
-template <int NB>
+template <int NB, int CK>
 cudaError_t launch_decode(const DecParams &dp, float *lse, float *scores, long long ld, cudaStream_t st) {
+    using S = SpSmem<NB, CK>;
     static bool attr = false;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(decode_full_mma<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SpSmem<NB>::bytes);
+        cudaError_t e = cudaFuncSetAttribute(decode_full_mma<NB, CK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)S::bytes);
         if (e != cudaSuccess) return e;
         attr = true;
     }
     const long long items = (long long)dp.sp.B * dp.sp.Hkv * dp.nchunk;
-    const long long blocks = (items + SpSmem<NB>::SW - 1) / SpSmem<NB>::SW;
+    const long long blocks = (items + S::SW - 1) / S::SW;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-    decode_full_mma<NB><<<(unsigned)blocks, SpSmem<NB>::SW * 32, SpSmem<NB>::bytes, st>>>(dp); count_launch();
+    decode_full_mma<NB, CK><<<(unsigned)blocks, S::SW * 32, S::bytes, st>>>(dp); count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     decode_combine<<<dim3(dp.sp.Hkv, dp.sp.B), 256, 0, st>>>(dp, lse, scores, ld); count_launch();
     return cudaGetLastError();
 }
 
-template <int NB>
+template <int NB, int CK>
 cudaError_t launch_nb(const SpParams &p, cudaStream_t st) {
+    using S = SpSmem<NB, CK>;
     static bool attr = false;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(sparse_attn_mma<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SpSmem<NB>::bytes);
+        cudaError_t e = cudaFuncSetAttribute(sparse_attn_mma<NB, CK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)S::bytes);
         if (e != cudaSuccess) return e;
         attr = true;
     }
     const long long items = (long long)p.B * p.Lq * p.Hkv;
-    const long long blocks = (items + SpSmem<NB>::SW - 1) / SpSmem<NB>::SW;
+    const long long blocks = (items + S::SW - 1) / S::SW;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-    sparse_attn_mma<NB><<<(unsigned)blocks, SpSmem<NB>::SW * 32, SpSmem<NB>::bytes, st>>>(p); count_launch();
+    sparse_attn_mma<NB, CK><<<(unsigned)blocks, S::SW * 32, S::bytes, st>>>(p); count_launch();
     return cudaGetLastError();
+}
+
+// Keys per chunk for 16-head groups (HYSPARSE_MMA_CHUNK=16|32 overrides).
+int chunk_keys_g16() {
+    const char *e = getenv("HYSPARSE_MMA_CHUNK");
+    if (e && strcmp(e, "32") == 0) return 32;
+    if (e && strcmp(e, "16") == 0) return 16;
+    return 32;
 }
 
 }  // namespace
@@ -591,7 +622,8 @@ cudaError_t sparse_attn_mma_launch(const Shape &s, const void *q, const void *k,
                    (__nv_bfloat16 *)out, (__nv_bfloat16 *)og, (__nv_bfloat16 *)ol, s.B, s.Lq, s.Lkv, s.Hq,
                    s.Hkv, s.G(), topk, window, s.scale * kLog2e, status, wait_ns, s.kv_len,
                    s.block_table, s.page_shift, s.max_pages, s.num_pages};
-    return s.G() <= 8 ? tc::launch_nb<1>(p, st) : tc::launch_nb<2>(p, st);
+    if (s.G() <= 8) return tc::launch_nb<1, 32>(p, st);
+    return tc::chunk_keys_g16() == 16 ? tc::launch_nb<2, 16>(p, st) : tc::launch_nb<2, 32>(p, st);
 }
 
 size_t decode_ws_bytes(const Shape &s) {
@@ -618,7 +650,9 @@ cudaError_t decode_full_mma_launch(const Shape &s, const void *q, const void *k,
     w += align_up(rows * nchunk * sizeof(float2), 256);
     dp.stash = reinterpret_cast<float *>(w);
     dp.nchunk = nchunk;
-    return s.G() <= 8 ? tc::launch_decode<1>(dp, lse, scores, ld, st) : tc::launch_decode<2>(dp, lse, scores, ld, st);
+    if (s.G() <= 8) return tc::launch_decode<1, 32>(dp, lse, scores, ld, st);
+    return tc::chunk_keys_g16() == 16 ? tc::launch_decode<2, 16>(dp, lse, scores, ld, st)
+                                      : tc::launch_decode<2, 32>(dp, lse, scores, ld, st);
 }
 
 }  // namespace hs
