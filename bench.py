@@ -175,17 +175,21 @@ def read_traffic(kernel_key: str, src_hash: str):
 
 def measure_l2(dev, mb: int = 64, passes: int = 8, reps: int = 5):
     """L2 read bandwidth on this GPU, measured live: the library's probe over
-    an L2-resident buffer of `mb` MiB (streaming 16-byte reads, and random
-    whole 256-byte rows as the sparse gather reads them), best of `reps`
-    timed calls after one untimed call that makes the buffer resident."""
+    an L2-resident buffer of `mb` MiB -- streaming 16-byte reads and random
+    whole 256-byte rows, each through registers (ld.global.cg, 4 CTAs of 512
+    threads per SM) and through cp.async into shared memory (one CTA of 7
+    warps per SM, as the row-gather kernel reads) -- best of `reps` timed calls
+    after one untimed call that makes the buffer resident.  The peak is the
+    best of the four."""
     import hybrid_sparse_attention_tcgen05_b200 as hs
-    props = torch.cuda.get_device_properties(dev)
-    blocks = props.multi_processor_count * 4
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     buf = torch.ones(mb << 20, dtype=torch.uint8, device=dev)
-    sink = torch.zeros(blocks, dtype=torch.int64, device=dev)
+    sink = torch.zeros(4 * sms, dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream(dev)
-    out = {"buffer_mib": mb, "passes_per_call": passes, "blocks": blocks, "threads_per_block": 512}
-    for mode, key in ((0, "stream_gbs"), (1, "row_gather_gbs")):
+    out = {"buffer_mib": mb, "passes_per_call": passes}
+    for mode, key in ((0, "stream_gbs"), (1, "row_gather_gbs"), (2, "cp_async_stream_gbs"),
+                      (3, "cp_async_row_gather_gbs")):
+        blocks = 4 * sms if mode < 2 else sms
         hs.probe_l2_read(buf, 1, mode, blocks, sink)
         best = 0.0
         for _ in range(reps):
@@ -197,7 +201,8 @@ def measure_l2(dev, mb: int = 64, passes: int = 8, reps: int = 5):
             torch.cuda.synchronize()
             best = max(best, passes * buf.numel() / (e0.elapsed_time(e1) / 1e3) / 1e9)
         out[key] = best
-    out["peak_gbs"] = max(out["stream_gbs"], out["row_gather_gbs"])
+    out["peak_gbs"] = max(out[k] for k in ("stream_gbs", "row_gather_gbs", "cp_async_stream_gbs",
+                                             "cp_async_row_gather_gbs"))
     del buf, sink
     return out
 

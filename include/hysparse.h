@@ -245,6 +245,9 @@ int hysparse_workspace_status(void *ws, hs_stream_t stream);
  *   mode 0: streaming 16-byte reads, `passes` times over the buffer;
  *   mode 1: whole 256-byte rows at hashed positions, passes * bytes / 256
  *           rows (the access pattern of the sparse layers' row gather).
+ *   modes 2 and 3: as 0 and 1, but through cp.async into shared memory
+ *           (one CTA of 7 warps per SM is the intended `blocks`: the path
+ *           and occupancy of the row-gather kernel); bytes >= 65536.
  * Either way passes * bytes bytes are read; time the call with events on
  * `stream`.  `sink` is a DEVICE array of at least `blocks` 64-bit words that
  * receives an XOR of what each CTA read (it keeps the loads live).
