@@ -249,7 +249,7 @@ def work_model(w):
 
 
 # kernel sources of the gather sparse layer (their hash keys the traffic record)
-SPARSE_GATHER_SRCS = ("sparse_mma.cu", "sparse_gather_tc.cu", "tc_util.cuh")
+SPARSE_GATHER_SRCS = ("sparse_mma.cu", "tc_util.cuh")
 
 
 def l2_served(w):
@@ -536,7 +536,7 @@ def bench_ours(args, w, ws_, rank, local):
         else:
             peak = peaks["hbm_gbs"]
             bound, peak_src = "hbm", None
-        roof = {"kernel": "sparse_attn (gather)", "bound": bound, "unit": "GB/s",
+        roof = {"kernel": "sparse_attn (gather: sparse_attn_mma)", "bound": bound, "unit": "GB/s",
                 "work": "(k_eff + w_eff) K and V rows per (row, kv head) + q, gate, out, idx"}
         if peak_src:
             roof["peak_source"] = peak_src
