@@ -70,6 +70,20 @@ __device__ __forceinline__ float ex2f(float x) {
 template <int NB>
 struct Branch {
     float m[NB][2], l[NB][2], o[NB][8][4];
+    // l holds this lane's share of each head column's row sum until finish()
+    // adds the eight lanes of the column (lanes with the same lane % 4)
+    __device__ void finish() {
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float x = l[nb][e];
+                x += __shfl_xor_sync(0xffffffffu, x, 4);
+                x += __shfl_xor_sync(0xffffffffu, x, 8);
+                x += __shfl_xor_sync(0xffffffffu, x, 16);
+                l[nb][e] = x;
+            }
+    }
     __device__ void init() {
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
@@ -157,16 +171,21 @@ __device__ __forceinline__ void issue_chunk(const SpParams &p, int entry, int po
     }
     vmask = __ballot_sync(0xffffffffu, key >= 0);
     const uint32_t sbase = smem_u32(stage);
-    const int half = lane >> 4, part = lane & 15;
+    // four rows per instruction: lanes 8q .. 8q+7 copy row 4 r4 + q, lane s
+    // its 16-byte chunk s in one instruction and chunk s + 8 in the next, so
+    // each instruction reads four whole 128-byte halves of rows
+    const int q = lane >> 3, sct = lane & 7;
 #pragma unroll
-    for (int r2 = 0; r2 < CK / 2; ++r2) {
-        const int row = 2 * r2 + half;
+    for (int r4 = 0; r4 < CK / 4; ++r4) {
+        const int row = 4 * r4 + q;
         const int kr = __shfl_sync(0xffffffffu, key, row);
         const bool ok = kr >= 0;
-        const size_t so = ok ? (size_t)kr * p.Hkv * 128 + part * 8 : 0;
-        const uint32_t d = sbase + sw_off(row, part);
-        cp_async16(d, kb + so, ok);
-        cp_async16(d + CK * RS, vb + so, ok);
+        const size_t so = ok ? (size_t)kr * p.Hkv * 128 + sct * 8 : 0;
+        const uint32_t d0 = sbase + sw_off(row, sct), d1 = sbase + sw_off(row, sct + 8);
+        cp_async16(d0, kb + so, ok);
+        cp_async16(d1, kb + so + 64, ok);
+        cp_async16(d0 + CK * RS, vb + so, ok);
+        cp_async16(d1 + CK * RS, vb + so + 64, ok);
     }
     cp_async_commit();
 }
@@ -240,9 +259,8 @@ __device__ __forceinline__ void compute_chunk(const uint8_t *stage, uint32_t vma
                     c[nb][mt][2 * rh + e] = pv;
                     ps += pv;
                 }
-            ps += __shfl_xor_sync(0xffffffffu, ps, 4);
-            ps += __shfl_xor_sync(0xffffffffu, ps, 8);
-            ps += __shfl_xor_sync(0xffffffffu, ps, 16);
+            // each lane keeps its own share of the row sum (same reference m
+            // across the head column); Branch::finish adds the shares up
             br.l[nb][e] = br.l[nb][e] * corr + ps;
             br.m[nb][e] = mn;
 #pragma unroll
@@ -331,6 +349,7 @@ __device__ __forceinline__ void run_branch(const WarpCtx &w, bool from_list, con
     }
     cp_async_wait<0>();
     __syncwarp();
+    br.finish();
 }
 
 template <int NB, int CK>
