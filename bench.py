@@ -271,7 +271,7 @@ def sparse_path_is_dense(w):
     tiles = sum(int((off + min(w.Lq, 128 * (t + 1)) - 1) // 128) + 1 for t in range((w.Lq + 127) // 128))
     per_tile = 2600.0 if (w.Hq // w.Hkv) % 2 == 0 else 4000.0
     dense_s = tiles * w.Hq * w.B * per_tile / (148.0 * 1.9e9)
-    gather_s = (sum_min(w, w.topk) + sum_min(w, w.window)) * w.Hkv * w.B * 512.0 / 6.0e12
+    gather_s = (sum_min(w, w.topk) + sum_min(w, w.window)) * w.Hkv * w.B * 512.0 / 12.0e12
     return dense_s < gather_s
 
 

@@ -98,7 +98,7 @@ __device__ __forceinline__ void cp16(uint32_t dst, const void *src) {
 __global__ void __launch_bounds__(kCpWarps * 32) l2_cp_probe(const uint8_t *buf, uint32_t nrows, long long steps,
                                                             int random, unsigned long long *sink) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, half = lane >> 4, part = lane & 15;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, q = lane >> 3, sct = lane & 7;
     const long long gw = (long long)blockIdx.x * kCpWarps + warp, nw = (long long)gridDim.x * kCpWarps;
     uint8_t *ring = smem + warp * kCpStages * kCpStage;
     // warp step s reads 32 rows: rows [32 s', 32 s' + 32) mod nrows (stream) or
@@ -107,9 +107,11 @@ __global__ void __launch_bounds__(kCpWarps * 32) l2_cp_probe(const uint8_t *buf,
     for (long long s0 = gw; s0 < steps; s0 += nw, ++k) {
         const uint32_t dst = (uint32_t)__cvta_generic_to_shared(ring + (k % kCpStages) * kCpStage);
         const uint32_t first = (uint32_t)((s0 * 32) % nrows);   // one 64-bit step per 32 rows
+        // the row gather's copy pattern: four rows per instruction, lanes
+        // 8q .. 8q+7 on row 4 r4 + q, lane s its 16-byte chunk s and then s + 8
 #pragma unroll
-        for (int r2 = 0; r2 < 16; ++r2) {
-            const uint32_t rl = 2 * r2 + half;
+        for (int r4 = 0; r4 < 8; ++r4) {
+            const uint32_t rl = 4 * r4 + q;
             uint32_t row;
             if (random) {
                 row = mix32(((uint32_t)s0 * 32u + rl) * 2654435761u + 12345u) % nrows;
@@ -117,7 +119,8 @@ __global__ void __launch_bounds__(kCpWarps * 32) l2_cp_probe(const uint8_t *buf,
                 row = first + rl;
                 if (row >= nrows) row -= nrows;
             }
-            cp16(dst + rl * 256 + part * 16, buf + (size_t)row * 256 + part * 16);
+            cp16(dst + rl * 256 + sct * 16, buf + (size_t)row * 256 + sct * 16);
+            cp16(dst + rl * 256 + (sct + 8) * 16, buf + (size_t)row * 256 + (sct + 8) * 16);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
         asm volatile("cp.async.wait_group %0;" ::"n"(kCpStages - 1) : "memory");
