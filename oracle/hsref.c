@@ -33,10 +33,17 @@
  *              sigma(x) = 1 / (1 + exp(-x))
  *   An empty global set (only possible with a caller-made index list of -1)
  *   gives Og = 0.
+ *   Own-window variant (the same section: the global branch computes "on the
+ *   shared KV cache", while the local branch "maintains a 128-token sliding
+ *   window"; read as: each sparse layer keeps its own K/V for its window):
+ *     Ol_h   = softmax attention of q'_h over { kw_j : pos-w+1 <= j <= pos }
+ *   with kw, vw the layer's own keys and values, stored for the last Lwin
+ *   positions of the sequence: buffer row r holds position Lkv - Lwin + r.
  *
  * Layouts (all row-major, C order):
  *   q_rows  [nrows][Hq][d]     float   the listed rows' queries
  *   k, v    [B][Lkv][Hkv][d]   float   the shared KV cache
+ *   kw, vw  [B][Lwin][Hkv][d]  float   a sparse layer's own window K/V (positions Lkv-Lwin ..)
  *   out     [nrows][Hq][d]     double
  *   lse     [nrows][Hq]        double
  *   scores  [nrows][Hkv][Lkv]  double  (entries j > pos are set to 0)
@@ -205,15 +212,27 @@ static int index_list_keys(const int *lst, int topk, int pos) {
 
 static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
 
-/* Sparse layer for the listed rows.  out_g / out_l may be NULL. */
-int hsref_sparse_rows(int B, int Lq, int Lkv, int Hq, int Hkv, int d, double scale,
-                      const float *q_rows, const float *k, const float *v,
-                      const int *row_b, const int *row_i, int nrows,
-                      const int *idx, int topk, const float *gate, int window,
-                      double *out, double *out_g, double *out_l) {
+/* Sparse layer for the listed rows; the window branch reads kw / vw (Lwin
+ * rows per batch element, positions Lkv - Lwin ..) when kw != NULL, else the
+ * shared cache.  out_g / out_l may be NULL. */
+static int sparse_rows_impl(int B, int Lq, int Lkv, int Hq, int Hkv, int d, double scale,
+                            const float *q_rows, const float *k, const float *v,
+                            const float *kw, const float *vw, int Lwin,
+                            const int *row_b, const int *row_i, int nrows,
+                            const int *idx, int topk, const float *gate, int window,
+                            double *out, double *out_g, double *out_l) {
     if (check_shape(B, Lq, Lkv, Hq, Hkv, d) || nrows < 0 || topk < 1 || window < 1) return -1;
     for (int r = 0; r < nrows; ++r)
         if (row_b[r] < 0 || row_b[r] >= B || row_i[r] < 0 || row_i[r] >= Lq) return -1;
+    const int woff = kw ? Lkv - Lwin : 0;   /* position of window-buffer row 0 */
+    if (kw) {
+        if (!vw || Lwin < 1 || Lwin > Lkv) return -1;
+        for (int r = 0; r < nrows; ++r) {
+            const int pos = Lkv - Lq + row_i[r];
+            const int lo = pos - window + 1 < 0 ? 0 : pos - window + 1;
+            if (lo < woff) return -1;        /* the window reaches below the buffer */
+        }
+    }
     const int G = Hq / Hkv;
     int err = 0;
 #pragma omp parallel for collapse(2) schedule(dynamic, 1)
@@ -244,13 +263,16 @@ int hsref_sparse_rows(int B, int Lq, int Lkv, int Hq, int Hkv, int d, double sca
                 int n = 0;
                 for (int t = 0; t < topk; ++t)
                     if (lst[t] != -1) keys_g[n++] = lst[t];
-                for (int t = 0; t < nl; ++t) keys_l[t] = lo + t;
+                for (int t = 0; t < nl; ++t) keys_l[t] = lo + t - woff;   /* rows of the window's buffer */
                 for (int hh = 0; hh < G; ++hh) {
                     const int h = g * G + hh;
                     const size_t o = ((size_t)r * Hq + h) * (size_t)d;
                     const float *q = q_rows + o;
                     attend_list(q, k, v, b, g, Lkv, Hkv, d, scale, keys_g, ng, s, og, NULL);
-                    attend_list(q, k, v, b, g, Lkv, Hkv, d, scale, keys_l, nl, s, ol, NULL);
+                    if (kw)
+                        attend_list(q, kw, vw, b, g, Lwin, Hkv, d, scale, keys_l, nl, s, ol, NULL);
+                    else
+                        attend_list(q, k, v, b, g, Lkv, Hkv, d, scale, keys_l, nl, s, ol, NULL);
                     double gs = sigmoid((double)gate[(size_t)r * Hq + h]);
                     for (int c = 0; c < d; ++c) {
                         if (out) out[o + c] = gs * og[c] + (1.0 - gs) * ol[c];
@@ -263,6 +285,28 @@ int hsref_sparse_rows(int B, int Lq, int Lkv, int Hq, int Hkv, int d, double sca
         }
     }
     return err;
+}
+
+int hsref_sparse_rows(int B, int Lq, int Lkv, int Hq, int Hkv, int d, double scale,
+                      const float *q_rows, const float *k, const float *v,
+                      const int *row_b, const int *row_i, int nrows,
+                      const int *idx, int topk, const float *gate, int window,
+                      double *out, double *out_g, double *out_l) {
+    return sparse_rows_impl(B, Lq, Lkv, Hq, Hkv, d, scale, q_rows, k, v, NULL, NULL, 0, row_b, row_i, nrows,
+                            idx, topk, gate, window, out, out_g, out_l);
+}
+
+/* The sparse layer with its own window K/V (kw, vw: [B][Lwin][Hkv][d],
+ * positions Lkv - Lwin .. Lkv - 1); every listed row's window must lie in it. */
+int hsref_sparse_rows_own_window(int B, int Lq, int Lkv, int Hq, int Hkv, int d, double scale,
+                                 const float *q_rows, const float *k, const float *v,
+                                 const float *kw, const float *vw, int Lwin,
+                                 const int *row_b, const int *row_i, int nrows,
+                                 const int *idx, int topk, const float *gate, int window,
+                                 double *out, double *out_g, double *out_l) {
+    if (!kw) return -1;
+    return sparse_rows_impl(B, Lq, Lkv, Hq, Hkv, d, scale, q_rows, k, v, kw, vw, Lwin, row_b, row_i, nrows,
+                            idx, topk, gate, window, out, out_g, out_l);
 }
 
 /* A whole hybrid block for the listed rows: the full layer, its top-k, then

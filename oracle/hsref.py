@@ -65,10 +65,12 @@ def _load():
         lib.hsref_topk_rows.argtypes = [P, LL, P, I, I, P]
         lib.hsref_sparse_rows.argtypes = [I, I, I, I, I, I, D, P, P, P, P, P, I, P, I, P, I,
                                           P, P, P]
+        lib.hsref_sparse_rows_own_window.argtypes = [I, I, I, I, I, I, D, P, P, P, P, P, I, P, P, I, P, I,
+                                                     P, I, P, P, P]
         lib.hsref_block_rows.argtypes = [I, I, I, I, I, I, D, P, P, P, P, P, I, I, P, P, I, I,
                                          P, P, P]
-        for f in ("hsref_full_rows", "hsref_topk_rows", "hsref_sparse_rows", "hsref_block_rows",
-                  "hsref_max_threads"):
+        for f in ("hsref_full_rows", "hsref_topk_rows", "hsref_sparse_rows", "hsref_sparse_rows_own_window",
+                  "hsref_block_rows", "hsref_max_threads"):
             getattr(lib, f).restype = I
         lib.hsref_set_threads.argtypes = [I]
         lib.hsref_set_threads.restype = None
@@ -148,10 +150,14 @@ def topk_rows(scores: torch.Tensor, n_valid, topk: int) -> torch.Tensor:
 
 
 def sparse_rows(q_rows: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rows, Lq: int, scale: float,
-                idx_rows: torch.Tensor, gate_rows: torch.Tensor, window: int):
+                idx_rows: torch.Tensor, gate_rows: torch.Tensor, window: int,
+                k_win: Optional[torch.Tensor] = None, v_win: Optional[torch.Tensor] = None):
     """One sparse layer for the listed rows.
 
     idx_rows [nrows,Hkv,topk] int32; gate_rows [nrows,Hq] fp32 logits.
+    k_win, v_win (optional, [B,Lwin,Hkv,d]): the layer's own window keys and
+    values for the last Lwin positions (row r = position Lkv - Lwin + r); the
+    window branch reads them instead of the shared cache.
     Returns (out, out_global, out_local), each [nrows,Hq,d] f64.
     """
     B, Lkv, Hkv, d = k.shape
@@ -164,6 +170,14 @@ def sparse_rows(q_rows: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rows, Lq
     out = torch.empty(nrows, Hq, d, dtype=torch.float64)
     og = torch.empty_like(out)
     ol = torch.empty_like(out)
+    if k_win is not None:
+        kwf, vwf = _f32(k_win), _f32(v_win)
+        rc = _load().hsref_sparse_rows_own_window(B, Lq, Lkv, Hq, Hkv, d, float(scale), _ptr(qf), _ptr(kf),
+                                                  _ptr(vf), _ptr(kwf), _ptr(vwf), int(kwf.shape[1]), _ptr(rb),
+                                                  _ptr(ri), nrows, _ptr(ix), int(topk), _ptr(gt), int(window),
+                                                  _ptr(out), _ptr(og), _ptr(ol))
+        _check(rc, "hsref_sparse_rows_own_window")
+        return out, og, ol
     rc = _load().hsref_sparse_rows(B, Lq, Lkv, Hq, Hkv, d, float(scale), _ptr(qf), _ptr(kf), _ptr(vf),
                                    _ptr(rb), _ptr(ri), nrows, _ptr(ix), int(topk), _ptr(gt),
                                    int(window), _ptr(out), _ptr(og), _ptr(ol))

@@ -240,6 +240,43 @@ def pin_sparse_branches_vs_sdpa():
     assert torch.allclose(ol, ref_l, atol=TOL, rtol=0), "local branch"
 
 
+def pin_own_window_branch_vs_sdpa():
+    """Own-window variant (each sparse layer keeps its own K/V for its window):
+    the local branch = torch attention over the band pos-w+1 .. pos with the
+    layer's own keys and values placed at their positions, for a buffer that
+    holds the whole sequence and for one that holds only its last Lwin
+    positions; the global branch still reads the shared cache unchanged."""
+    B, Lkv, Hq, Hkv, d = 2, 16, 4, 2, 8
+    scale = 1.0 / math.sqrt(d)
+    window, topk = 4, 5
+    for Lq, Lwin in ((16, 16), (3, 6)):
+        q, k, v, gate = _sparse_case(700 + Lq, B, Lq, Lkv, Hq, Hkv, d)
+        kw = _rand(B, Lwin, Hkv, d, seed=710 + Lq)
+        vw = _rand(B, Lwin, Hkv, d, seed=720 + Lq)
+        rows = _all_rows(B, Lq)
+        rng = np.random.default_rng(7)
+        sets = [[rng.choice(Lkv - Lq + i + 1, size=min(topk, Lkv - Lq + i + 1), replace=False).tolist()
+                 for _ in range(Hkv)] for (_, i) in rows]
+        idx = _idx_from_sets(sets, topk)
+        qr, gr = _q_rows(q, rows), _q_rows(gate, rows)
+        out, og, ol = oracle.sparse_rows(qr, k, v, rows, Lq, scale, idx, gr, window, k_win=kw, v_win=vw)
+        out0, og0, _ = oracle.sparse_rows(qr, k, v, rows, Lq, scale, idx, gr, window)
+        assert torch.equal(og, og0), "global branch reads the shared cache"
+        kfull = torch.zeros(B, Lkv, Hkv, d)
+        vfull = torch.zeros(B, Lkv, Hkv, d)
+        kfull[:, Lkv - Lwin:] = kw
+        vfull[:, Lkv - Lwin:] = vw
+        i = torch.arange(Lq)[:, None]
+        j = torch.arange(Lkv)[None, :]
+        pos = Lkv - Lq + i
+        band = (j <= pos) & (j >= pos - window + 1)
+        ref_l = _sdpa(q, kfull, vfull, band, scale).reshape(B * Lq, Hq, d)
+        assert torch.allclose(ol, ref_l, atol=TOL, rtol=0), "own-window local branch"
+        sg = torch.sigmoid(gr.double())[..., None]
+        assert torch.allclose(out, sg * og + (1 - sg) * ol, atol=TOL, rtol=0), "gate"
+        assert not torch.allclose(ol, _sdpa(q, k, v, band, scale).reshape(B * Lq, Hq, d))
+
+
 def pin_sparse_reduces_to_full():
     """With k >= pos+1 the global branch is full causal attention; with a
     window >= Lkv the local branch is full causal attention."""
@@ -305,6 +342,7 @@ ALL_PINS = [
     pin_topk_matches_stable_argsort,
     pin_topk_bruteforce,
     pin_sparse_branches_vs_sdpa,
+    pin_own_window_branch_vs_sdpa,
     pin_sparse_reduces_to_full,
     pin_gate_limits,
     pin_block_composes,

@@ -50,3 +50,16 @@ def test_bad_shapes_rejected():
         oracle.full_rows(torch.randn(1, 4, 4), k, k, [(0, 9)], 8, 0.5)   # row out of range
     with pytest.raises(ValueError):
         oracle.full_rows(torch.randn(1, 4, 4), k, k, [(0, 0)], 9, 0.5)   # Lq > Lkv
+
+
+def test_own_window_buffer_must_cover_every_window():
+    """The own-window variant reads positions Lkv - Lwin .. Lkv - 1 only: a row
+    whose window starts below that is an argument error, not a silent read."""
+    k = torch.randn(1, 8, 1, 4)
+    q = torch.randn(1, 1, 4)
+    idx = torch.full((1, 1, 2), -1, dtype=torch.int32)
+    kw = torch.randn(1, 3, 1, 4)
+    # row 0 of Lq = 1: pos 7, window 3 -> keys 5..7, inside a 3-row tail buffer
+    oracle.sparse_rows(q, k, k, [(0, 0)], 1, 0.5, idx, torch.zeros(1, 1), 3, k_win=kw, v_win=kw)
+    with pytest.raises(ValueError):   # window 4 reaches key 4, below the buffer
+        oracle.sparse_rows(q, k, k, [(0, 0)], 1, 0.5, idx, torch.zeros(1, 1), 4, k_win=kw, v_win=kw)
