@@ -29,7 +29,7 @@ from ._lib import HysparseError, HsShape
 
 __all__ = ["shape_of", "workspace_size", "alloc_workspace", "full_attn_scores", "topk",
            "sparse_attn", "block", "block_paged", "workspace_status", "version", "launch_count",
-           "HysparseError", "HsShape"]
+           "kv_cache_bytes", "HysparseError", "HsShape"]
 
 
 def _dtype_code(t: torch.dtype) -> int:
@@ -139,10 +139,17 @@ def topk(q_shape: HsShape, scores: torch.Tensor, k_top: int, *, row_begin: int =
 def sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor,
                 gate_logit: torch.Tensor, window: int, *, want_branches: bool = False,
                 out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
-                scale: Optional[float] = None):
+                scale: Optional[float] = None, k_win: Optional[torch.Tensor] = None,
+                v_win: Optional[torch.Tensor] = None):
     """One sparse layer.  Returns out, or (out, out_global, out_local) when
-    want_branches."""
-    dev = _need_cuda(q, k, v, idx, gate_logit, out, ws)
+    want_branches.
+
+    k_win / v_win ([B, lwin, Hkv, d], the layer's own window keys and values
+    for cache positions Lkv - lwin .. Lkv - 1): the local branch reads them
+    instead of k / v (hysparse_sparse_attn_own_window)."""
+    dev = _need_cuda(q, k, v, idx, gate_logit, out, ws, k_win, v_win)
+    if (k_win is None) != (v_win is None):
+        raise ValueError("k_win and v_win go together")
     if idx.dtype != torch.int32 or gate_logit.dtype != torch.float32:
         raise TypeError("idx must be int32 and gate_logit float32")
     s = shape_of(q, k, scale)
@@ -153,6 +160,18 @@ def sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Te
     ol = torch.empty_like(q) if want_branches else None
     if ws is None:
         ws = alloc_workspace(s, k_top, window, 1, 1, dev)
+    if k_win is not None:
+        lwin = k_win.shape[1]
+        want = (k.shape[0], lwin) + tuple(k.shape[2:])
+        for t in (k_win, v_win):
+            if tuple(t.shape) != want or t.dtype != k.dtype or not t.is_contiguous():
+                raise TypeError("k_win and v_win must be contiguous [B, lwin, Hkv, d] of k's dtype")
+        st = _lib.lib().hysparse_sparse_attn_own_window(
+            ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(k_win), _ptr(v_win), int(lwin), _ptr(idx),
+            int(k_top), _ptr(gate_logit), int(window), _ptr(out), _ptr(og), _ptr(ol), _ptr(ws), ws.numel(),
+            _stream(dev))
+        _lib.check(st, "hysparse_sparse_attn_own_window")
+        return (out, og, ol) if want_branches else out
     st = _lib.lib().hysparse_sparse_attn(
         ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), int(k_top), _ptr(gate_logit),
         int(window), _ptr(out), _ptr(og), _ptr(ol), _ptr(ws), ws.numel(), _stream(dev))
@@ -276,6 +295,27 @@ def probe_l2_read(buf: torch.Tensor, passes: int, mode: int, blocks: int, sink: 
     st = _lib.lib().hysparse_probe_l2_read(_ptr(buf), nbytes, int(passes), int(mode), int(blocks), _ptr(sink),
                                            _stream(dev))
     _lib.check(st, "hysparse_probe_l2_read")
+
+
+def kv_cache_bytes(B: int, Lkv: int, Hkv: int, d: int, elem_bytes: int, n_sparse: int, window: int,
+                   own_window: bool = False, Lq: int = 1) -> dict:
+    """KV-cache bytes one hybrid block keeps for a batch (HySparse abstract and
+    write-up section 3.1: only the full layer writes a cache, which its sparse
+    layers reuse; section 2.2: a sparse layer's local branch may keep its own
+    sliding window).
+
+    full: the full layer's K and V, 2 * B * Lkv * Hkv * d elements.
+    sparse: 0 when the sparse layers read the shared cache; with own windows,
+    each of the n_sparse layers keeps K and V for the rows its window branch
+    reads while Lq new rows are processed, min(Lkv, window - 1 + Lq) per
+    sequence (window rows for one decode step).
+    dense_equivalent: the same 1 + n_sparse layers all with full caches.
+    """
+    per_row = 2 * B * Hkv * d * elem_bytes
+    full = per_row * Lkv
+    sparse = n_sparse * per_row * min(Lkv, window - 1 + Lq) if own_window else 0
+    return {"full": full, "sparse": sparse, "total": full + sparse,
+            "dense_equivalent": (1 + n_sparse) * full}
 
 
 def launch_count() -> int:

@@ -28,6 +28,7 @@ EXPORTS = (
     "hysparse_full_attn_scores",
     "hysparse_topk",
     "hysparse_sparse_attn",
+    "hysparse_sparse_attn_own_window",
     "hysparse_block",
     "hysparse_block_varlen",
     "hysparse_block_paged",
@@ -75,6 +76,8 @@ def lib():
     L.hysparse_topk.restype = I
     L.hysparse_sparse_attn.argtypes = [SP, P, P, P, P, I, P, I, P, P, P, P, SZ, P]
     L.hysparse_sparse_attn.restype = I
+    L.hysparse_sparse_attn_own_window.argtypes = [SP, P, P, P, P, P, I, P, I, P, I, P, P, P, P, SZ, P]
+    L.hysparse_sparse_attn_own_window.restype = I
     L.hysparse_block.argtypes = [SP, P, P, P, P, P, I, P, P, P, I, I, P, I, P, SZ, P]
     L.hysparse_block.restype = I
     L.hysparse_block_varlen.argtypes = [SP, P, P, P, P, P, P, I, P, P, P, I, I, P, P, SZ, P]

@@ -861,10 +861,20 @@ cudaError_t sparse_pair_tc_launch(const Shape &s, const void *q, const void *k, 
                                   int window, void *out, void *og, void *ol, const uint32_t *mask, int W,
                                   uint32_t *wl, unsigned int *status, unsigned long long wait_ns, cudaStream_t st) {
     using namespace tc;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mkw, mvw;
     if (!make_map(&mq, q, s.Hq, s.Lq, s.B) || !make_map(&mk, k, s.Hkv, s.Lkv, s.B) ||
         !make_map(&mv, v, s.Hkv, s.Lkv, s.B))
         return cudaErrorInvalidValue;
+    // a layer with its own window K/V (one row per cache position, so the
+    // same [B][Lkv][Hkv][d] extent) reads the window pass from that buffer
+    if (s.k_win != nullptr) {
+        if (s.Lwin != s.Lkv || !make_map(&mkw, s.k_win, s.Hkv, s.Lkv, s.B) ||
+            !make_map(&mvw, s.v_win, s.Hkv, s.Lkv, s.B))
+            return cudaErrorInvalidValue;
+    } else {
+        mkw = mk;
+        mvw = mv;
+    }
     static bool attr_done = false;
     if (!attr_done) {
         cudaError_t e = fwd_prepare<FWD_WIN>();
@@ -881,7 +891,7 @@ cudaError_t sparse_pair_tc_launch(const Shape &s, const void *q, const void *k, 
     fp.window = window; fp.W = W; fp.selmask = mask; fp.wl = wl; fp.gate = gate;
     fp.out_g = (__nv_bfloat16 *)og; fp.out_l = (__nv_bfloat16 *)ol;
     const int n_tiles = (s.Lq + BM - 1) / BM;
-    attn_fwd_tc<FWD_WIN><<<tile_grid(s.Hq / 2, n_tiles, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp); count_launch();
+    attn_fwd_tc<FWD_WIN><<<tile_grid(s.Hq / 2, n_tiles, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mkw, mvw, fp); count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     attn_fwd_tc<FWD_SEL><<<tile_grid(s.Hq / 2, n_tiles, s.B), FWD_THREADS, kFwdSmem, st>>>(mq, mk, mv, fp); count_launch();

@@ -126,6 +126,9 @@ constexpr double kPairTileCycles = 2600.0;       // paired-head pipeline (even G
 constexpr double kGatherBytesPerS = 12.0e12;   // measured 11.9-15.6 TB/s of gathered rows (prefill)
 bool prefer_dense_sparse(const Shape &s, int topk, int window) {
     if (!sparse_dense_supported(s)) return false;
+    // own window K/V: only the paired-head pipeline reads the window pass from
+    // a second buffer, and only one that spans the whole cache
+    if (s.k_win != nullptr && (s.Lwin != s.Lkv || !sparse_pair_supported(s))) return false;
     const char *e = getenv("HYSPARSE_SPARSE_PATH");
     if (e && strcmp(e, "dense") == 0) return true;
     if (e && strcmp(e, "gather") == 0) return false;
@@ -151,7 +154,7 @@ bool prefer_dense_sparse(const Shape &s, int topk, int window) {
 // (sparse_gather_tc.cu) or the warp-MMA one (sparse_mma.cu).
 // HYSPARSE_GATHER_KERNEL=tc|mma overrides the default.
 bool use_gather_tc(const Shape &s) {
-    if (!sparse_gather_tc_supported(s)) return false;
+    if (!sparse_gather_tc_supported(s) || s.k_win != nullptr) return false;
     const char *e = getenv("HYSPARSE_GATHER_KERNEL");
     if (e && strcmp(e, "tc") == 0) return true;
     return false;
@@ -240,6 +243,28 @@ int hysparse_topk(const hs_shape *shape, const float *scores, long long ld_score
     return run_topk(s, scores, ld_scores, row_begin, row_count, topk, idx, (cudaStream_t)stream);
 }
 
+}  // extern "C"
+
+namespace {
+// Checks and runs one sparse layer for hysparse_sparse_attn and
+// hysparse_sparse_attn_own_window (s carries the own window buffer, if any).
+int sparse_attn_impl(const Shape &s, const void *q, const void *k, const void *v, const int32_t *idx, int topk,
+                     const float *gate_logit, int window, void *out, void *out_global, void *out_local, void *ws,
+                     size_t ws_bytes, cudaStream_t st) {
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(gate_logit) ||
+        !aligned16(out))
+        return HS_ERR_INVALID_ARG;
+    if ((out_global && !aligned16(out_global)) || (out_local && !aligned16(out_local)))
+        return HS_ERR_INVALID_ARG;
+    if (topk < 1 || topk > kMaxTopk || window < 1 || window > kMaxWindow) return HS_ERR_INVALID_ARG;
+    if (!aligned16(ws)) return HS_ERR_INVALID_ARG;
+    if (ws_bytes < ws_layout(s, topk, 1).sparse_end) return HS_ERR_WORKSPACE;
+    return run_sparse(s, q, k, v, idx, topk, gate_logit, window, out, out_global, out_local, ws, st);
+}
+}  // namespace
+
+extern "C" {
+
 int hysparse_sparse_attn(const hs_shape *shape, const void *q, const void *k, const void *v,
                          const int32_t *idx, int topk, const float *gate_logit, int window,
                          void *out, void *out_global, void *out_local, void *ws, size_t ws_bytes,
@@ -247,16 +272,28 @@ int hysparse_sparse_attn(const hs_shape *shape, const void *q, const void *k, co
     Shape s;
     int rc = resolve_shape(shape, &s);
     if (rc != HS_OK) return rc;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) ||
-        !aligned16(gate_logit) || !aligned16(out))
-        return HS_ERR_INVALID_ARG;
-    if ((out_global && !aligned16(out_global)) || (out_local && !aligned16(out_local)))
-        return HS_ERR_INVALID_ARG;
-    if (topk < 1 || topk > kMaxTopk || window < 1 || window > kMaxWindow) return HS_ERR_INVALID_ARG;
-    if (!aligned16(ws)) return HS_ERR_INVALID_ARG;
-    if (ws_bytes < ws_layout(s, topk, 1).sparse_end) return HS_ERR_WORKSPACE;
-    return run_sparse(s, q, k, v, idx, topk, gate_logit, window, out, out_global, out_local, ws,
-                      (cudaStream_t)stream);
+    return sparse_attn_impl(s, q, k, v, idx, topk, gate_logit, window, out, out_global, out_local, ws, ws_bytes,
+                            (cudaStream_t)stream);
+}
+
+int hysparse_sparse_attn_own_window(const hs_shape *shape, const void *q, const void *k, const void *v,
+                                    const void *k_win, const void *v_win, int lwin, const int32_t *idx, int topk,
+                                    const float *gate_logit, int window, void *out, void *out_global,
+                                    void *out_local, void *ws, size_t ws_bytes, hs_stream_t stream) {
+    Shape s;
+    int rc = resolve_shape(shape, &s);
+    if (rc != HS_OK) return rc;
+    if (!aligned16(k_win) || !aligned16(v_win) || lwin < 1 || lwin > s.Lkv) return HS_ERR_INVALID_ARG;
+    if (window < 1 || window > kMaxWindow) return HS_ERR_INVALID_ARG;
+    // the buffer holds positions Lkv - lwin .. Lkv - 1 and must reach back to
+    // the first key of the first query row's window
+    const int first_key = s.Lkv - s.Lq - window + 1 > 0 ? s.Lkv - s.Lq - window + 1 : 0;
+    if (s.Lkv - lwin > first_key) return HS_ERR_INVALID_ARG;
+    s.k_win = k_win;
+    s.v_win = v_win;
+    s.Lwin = lwin;
+    return sparse_attn_impl(s, q, k, v, idx, topk, gate_logit, window, out, out_global, out_local, ws, ws_bytes,
+                            (cudaStream_t)stream);
 }
 
 namespace {

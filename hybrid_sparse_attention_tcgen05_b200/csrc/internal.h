@@ -28,6 +28,11 @@ struct Shape {
     // contiguous [B][Lkv][Hkv][d] caches.
     const int32_t *block_table = nullptr;
     int page_shift = 0, max_pages = 0, num_pages = 0;
+    // a sparse layer's own window K/V (hysparse_sparse_attn_own_window):
+    // [B][Lwin][Hkv][d] holding positions Lkv - Lwin .. Lkv - 1; the window
+    // branch reads it instead of k, v.  NULL: the shared cache.
+    const void *k_win = nullptr, *v_win = nullptr;
+    int Lwin = 0;
     int G() const { return Hq / Hkv; }
 };
 

@@ -190,7 +190,8 @@ __global__ void __launch_bounds__(1024)
 sparse_attn_simt(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                  const int32_t *__restrict__ idx, int topk, const float *__restrict__ gate,
                  int window, T *__restrict__ out, T *__restrict__ out_g, T *__restrict__ out_l,
-                 int Lq, int Lkv, int Hq, int Hkv, float scale_log2, unsigned int *status) {
+                 int Lq, int Lkv, int Hq, int Hkv, float scale_log2, unsigned int *status,
+                 const T *__restrict__ kw, const T *__restrict__ vw, int Lwin) {
     extern __shared__ float smem[];
     const int G = Hq / Hkv;
     float *Ks = smem;
@@ -215,7 +216,12 @@ sparse_attn_simt(const T *__restrict__ q, const T *__restrict__ k, const T *__re
     attend_keys<T, D>(kbase, vbase, Hkv, list, topk, true, 0, pos, qs, Ks, Vs, ps, keys,
                       scale_log2, sg, status);
     const int lo = max(0, pos - window + 1);
-    attend_keys<T, D>(kbase, vbase, Hkv, nullptr, pos - lo + 1, false, lo, pos, qs, Ks, Vs, ps,
+    // the window branch: the shared cache, or the layer's own window K/V whose
+    // row 0 is position Lkv - Lwin (the keys are then that buffer's rows)
+    const int woff = kw ? Lkv - Lwin : 0;
+    const T *kwb = kw ? kw + ((size_t)b * Lwin * Hkv + g) * D : kbase;
+    const T *vwb = kw ? vw + ((size_t)b * Lwin * Hkv + g) * D : vbase;
+    attend_keys<T, D>(kwb, vwb, Hkv, nullptr, pos - lo + 1, false, lo - woff, pos - woff, qs, Ks, Vs, ps,
                       keys, scale_log2, sl, status);
 
     const float x = gate[((size_t)b * Lq + i) * Hq + h];
@@ -261,7 +267,8 @@ cudaError_t launch_sparse_simt(const Shape &s, const void *q, const void *k, con
     dim3 grid(s.Lq, s.Hkv, s.B);
     kern<<<grid, 32 * G, sm, st>>>((const T *)q, (const T *)k, (const T *)v, idx, topk, gate,
                                    window, (T *)out, (T *)og, (T *)ol, s.Lq, s.Lkv, s.Hq, s.Hkv,
-                                   s.scale * kLog2e, status); count_launch();
+                                   s.scale * kLog2e, status, (const T *)s.k_win, (const T *)s.v_win,
+                                   s.Lwin); count_launch();
     return cudaGetLastError();
 }
 

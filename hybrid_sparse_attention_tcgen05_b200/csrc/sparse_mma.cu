@@ -30,9 +30,7 @@ namespace hs {
 namespace tc {
 namespace {
 
-constexpr int RS = 256;
-// Stages of the 8-head configuration (3 with 4 warps, or 2 with 7 warps).
-constexpr int mma_stages_g8() { return 2; }           // row stride in shared memory (bytes): one K or V row
+constexpr int RS = 256;           // row stride in shared memory (bytes): one K or V row
 
 // Byte offset of 16-byte chunk c16 (0..15) of row r of a staged tile: the
 // chunks of a row are XOR-permuted by r mod 8, so the eight rows an ldmatrix
@@ -42,8 +40,9 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c16) {
     return (uint32_t)r * RS + ((uint32_t)(c16 ^ (r & 7)) << 4);
 }
 
-// Per head-block count NB (heads padded to 8*NB) and keys per chunk CK (16
-// or 32): SW warps (items) per CTA, each with an ST-stage chunk ring.  A
+// Per head-block count NB (heads padded to 8*NB) and keys per chunk CK (32;
+// 16 measured slower): SW warps (items) per CTA, each with an ST-stage chunk
+// ring.  A
 // warp stages its query rows (and, at the end, its output rows) in the ring's
 // last stage, which the pipeline only fills after the rows are in registers.
 // Measured at the 64k-token, 16-head workload: 32-key chunks, two stages,
@@ -51,8 +50,8 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c16) {
 // gather stream; more of them keep more bytes in flight).
 template <int NB, int CK>
 struct SpSmem {
-    static constexpr int ST = NB == 1 ? mma_stages_g8() : (CK == 16 ? 4 : 2);
-    static constexpr int SW = NB == 1 ? (ST == 3 ? 4 : 7) : (CK == 16 ? 6 : 7);
+    static constexpr int ST = 2;
+    static constexpr int SW = 7;
     static constexpr int STAGE_BYTES = 2 * CK * RS;
     static constexpr int WARP_BYTES = ST * STAGE_BYTES;
     static constexpr size_t bytes = (size_t)SW * WARP_BYTES;
@@ -112,6 +111,10 @@ struct SpParams {
     // block_table[b * max_pages + (j >> page_shift)].  NULL: contiguous caches.
     const int32_t *block_table;
     int page_shift, max_pages, num_pages;
+    // the layer's own window K/V ([B][Lwin][Hkv][128], row 0 = position
+    // Lkv - Lwin) read by the window branch, or NULL: the shared cache
+    const __nv_bfloat16 *kw = nullptr, *vw = nullptr;
+    int Lwin = 0;
 };
 
 // Cache length of sequence b: kv_len[b] when given (a value outside
@@ -404,7 +407,20 @@ __global__ void __launch_bounds__(SpSmem<NB, CK>::SW * 32, 1) sparse_attn_mma(co
     w.c2 = p.scale_log2;
     Branch<NB> bg, bl;
     run_branch<NB, CK>(w, true, bq, bg);
-    run_branch<NB, CK>(w, false, bq, bl);
+    if (p.kw != nullptr) {
+        // the window branch over the layer's own window K/V: its keys are that
+        // buffer's rows, position - (Lkv - Lwin)
+        const int off = p.Lkv - p.Lwin;
+        WarpCtx wl = w;
+        wl.kb = p.kw + ((size_t)b * p.Lwin * p.Hkv + g) * 128;
+        wl.vb = p.vw + ((size_t)b * p.Lwin * p.Hkv + g) * 128;
+        wl.table = nullptr;
+        wl.lo = w.lo - off;
+        wl.pos = w.pos - off;
+        run_branch<NB, CK>(wl, false, bq, bl);
+    } else {
+        run_branch<NB, CK>(w, false, bq, bl);
+    }
 
     // gate merge, stage the G output rows in shared memory, write them once
     __syncwarp();
@@ -620,14 +636,6 @@ cudaError_t launch_nb(const SpParams &p, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-// Keys per chunk for 16-head groups (HYSPARSE_MMA_CHUNK=16|32 overrides).
-int chunk_keys_g16() {
-    const char *e = getenv("HYSPARSE_MMA_CHUNK");
-    if (e && strcmp(e, "32") == 0) return 32;
-    if (e && strcmp(e, "16") == 0) return 16;
-    return 32;
-}
-
 }  // namespace
 }  // namespace tc
 
@@ -641,8 +649,11 @@ cudaError_t sparse_attn_mma_launch(const Shape &s, const void *q, const void *k,
                    (__nv_bfloat16 *)out, (__nv_bfloat16 *)og, (__nv_bfloat16 *)ol, s.B, s.Lq, s.Lkv, s.Hq,
                    s.Hkv, s.G(), topk, window, s.scale * kLog2e, status, wait_ns, s.kv_len,
                    s.block_table, s.page_shift, s.max_pages, s.num_pages};
+    p.kw = (const __nv_bfloat16 *)s.k_win;
+    p.vw = (const __nv_bfloat16 *)s.v_win;
+    p.Lwin = s.Lwin;
     if (s.G() <= 8) return tc::launch_nb<1, 32>(p, st);
-    return tc::chunk_keys_g16() == 16 ? tc::launch_nb<2, 16>(p, st) : tc::launch_nb<2, 32>(p, st);
+    return tc::launch_nb<2, 32>(p, st);
 }
 
 size_t decode_ws_bytes(const Shape &s) {
@@ -670,8 +681,7 @@ cudaError_t decode_full_mma_launch(const Shape &s, const void *q, const void *k,
     dp.stash = reinterpret_cast<float *>(w);
     dp.nchunk = nchunk;
     if (s.G() <= 8) return tc::launch_decode<1, 32>(dp, lse, scores, ld, st);
-    return tc::chunk_keys_g16() == 16 ? tc::launch_decode<2, 16>(dp, lse, scores, ld, st)
-                                      : tc::launch_decode<2, 32>(dp, lse, scores, ld, st);
+    return tc::launch_decode<2, 32>(dp, lse, scores, ld, st);
 }
 
 }  // namespace hs

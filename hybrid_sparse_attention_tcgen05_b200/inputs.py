@@ -144,6 +144,47 @@ def make_inputs(w: Workload, seed: int = 0, device: str = "cpu") -> Dict[str, ob
     return res
 
 
+def make_window_kv(w: Workload, lwin: int, seed: int = 0, device: str = "cpu"):
+    """Draw one sparse layer's own window keys and values, [B,lwin,Hkv,d]
+    each in the workload dtype, for cache positions Lkv - lwin .. Lkv - 1.
+
+    Drawn from a generator of their own (so the block's other inputs are the
+    same with or without them): standard normal for the "normal" recipe,
+    normal with std 1/sqrt(d) for the "shifted" one (the scale of that
+    recipe's unshifted keys and values).
+    """
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    sigma = 1.0 / math.sqrt(w.d) if w.dist == "shifted" else 1.0
+    kw = torch.randn(w.B, lwin, w.Hkv, w.d, generator=g, device=dev, dtype=torch.float32) * sigma
+    vw = torch.randn(w.B, lwin, w.Hkv, w.d, generator=g, device=dev, dtype=torch.float32) * sigma
+    return kw.to(torch_dtype(w)), vw.to(torch_dtype(w))
+
+
+def random_index_sets(B: int, Hkv: int, Lq: int, Lkv: int, topk: int, seed: int = 0) -> torch.Tensor:
+    """Seeded index sets for a sparse layer, int32 [B,Hkv,Lq,topk] on the
+    host: row i of (b, g) holds min(pos(i) + 1, topk) distinct keys drawn
+    uniformly from [0, pos(i)], pos(i) = Lkv - Lq + i, in ascending order,
+    padded with -1 (the layout a top-k selection writes)."""
+    g = torch.Generator().manual_seed(seed)
+    idx = torch.full((B, Hkv, Lq, topk), -1, dtype=torch.int32)
+    for b in range(B):
+        for h in range(Hkv):
+            for i in range(Lq):
+                n = Lkv - Lq + i + 1
+                take = min(n, topk)
+                if n <= 4 * topk:
+                    pick = torch.randperm(n, generator=g)[:take]
+                else:
+                    pick = torch.unique(torch.randint(0, n, (2 * take,), generator=g))
+                    while pick.numel() < take:
+                        pick = torch.unique(torch.cat([pick, torch.randint(0, n, (take,), generator=g)]))
+                    pick = pick[torch.randperm(pick.numel(), generator=g)[:take]]
+                idx[b, h, i, :take] = pick.sort().values.to(torch.int32)
+    return idx
+
+
 def sample_rows(Lq: int, topk: int, window: int, n_random: int = 256, seed: int = 0,
                 edge: int = 64) -> List[int]:
     """A seeded, sorted sample of query rows for checks at full size.
@@ -177,5 +218,5 @@ def workload(name: str, **override) -> Workload:
     return w.with_(**override) if override else w
 
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "sample_rows", "to_oracle_f32",
-           "torch_dtype", "workload", "n_shift_keys"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_window_kv", "random_index_sets", "sample_rows",
+           "to_oracle_f32", "torch_dtype", "workload", "n_shift_keys"]

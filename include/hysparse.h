@@ -141,6 +141,31 @@ int hysparse_sparse_attn(const hs_shape *shape, const void *q, const void *k, co
                          void *out, void *out_global, void *out_local, void *ws, size_t ws_bytes,
                          hs_stream_t stream);
 
+/* One sparse layer whose local branch reads the layer's own window K/V
+ * (write-up section 2.2: the global branch computes on the KV cache that the
+ * full layer shares, while the local branch maintains its own 128-token
+ * sliding window).  Same computation, arguments and errors as
+ * hysparse_sparse_attn, except that the local branch's keys and values come
+ * from k_win / v_win instead of k / v:
+ *   Ol = softmax attention of q[b,i,h] over
+ *        { k_win[b, j - (Lkv - lwin)] : max(0, pos(i)-window+1) <= j <= pos(i) }
+ *   with values v_win at the same rows.
+ * k_win, v_win  [B][lwin][Hkv][d] (dtype of the shape, caller-owned, 16-byte
+ * aligned): the layer's window keys and values for cache positions
+ * Lkv - lwin .. Lkv - 1 (lwin = Lkv for a prefill that projects every
+ * position; lwin = window - 1 + Lq, or any length that reaches back far
+ * enough, for decode against a ring of the last tokens laid out in position
+ * order).  1 <= lwin <= Lkv and Lkv - lwin <= max(0, Lkv - Lq - window + 1)
+ * (the buffer covers the first row's window), else HS_ERR_INVALID_ARG.
+ * The global branch still reads k and v with idx.  Passing k_win = k,
+ * v_win = v, lwin = Lkv gives hysparse_sparse_attn's result, bit for bit
+ * when Hq / Hkv is even (with an odd ratio the plain call may choose a
+ * kernel that this one does not, and the two agree to rounding). */
+int hysparse_sparse_attn_own_window(const hs_shape *shape, const void *q, const void *k, const void *v,
+                                    const void *k_win, const void *v_win, int lwin, const int32_t *idx, int topk,
+                                    const float *gate_logit, int window, void *out, void *out_global,
+                                    void *out_local, void *ws, size_t ws_bytes, hs_stream_t stream);
+
 /* A whole hybrid block (HySparse abstract: one full layer interleaved with
  * several sparse layers; write-up section 3.1: index sharing and cache reuse):
  * the full layer over all rows (out_full, and its LSE into `lse` when not

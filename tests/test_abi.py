@@ -133,6 +133,30 @@ def test_sparse_attn_rejects(L):
     assert f(s=shape(dtype=_lib.HS_BF16, d=64)) == _lib.HS_ERR_UNSUPPORTED
 
 
+def test_sparse_attn_own_window_rejects(L):
+    """The own window buffer must be aligned, hold 1 .. Lkv rows and reach
+    back to the first key of the first query row's window."""
+    def f(s=None, kw=P(8), vw=P(9), lwin=None, w=16, q=P(1), wsb=None):
+        s = s or shape()
+        lwin = s.Lkv if lwin is None else lwin
+        wsb = ws_size(L, s) if wsb is None else wsb
+        return L.hysparse_sparse_attn_own_window(ctypes.byref(s), q, P(2), P(3), kw, vw, lwin, P(4), 8, P(5), w,
+                                                 P(6), None, None, P(7), wsb, None)
+    assert f(kw=None) == _lib.HS_ERR_INVALID_ARG
+    assert f(vw=None) == _lib.HS_ERR_INVALID_ARG
+    assert f(vw=ctypes.c_void_p(A + 8)) == _lib.HS_ERR_INVALID_ARG
+    assert f(lwin=0) == _lib.HS_ERR_INVALID_ARG
+    assert f(lwin=65) == _lib.HS_ERR_INVALID_ARG
+    assert f(lwin=63) == _lib.HS_ERR_INVALID_ARG           # prefill: row 0 sees key 0
+    dec = shape(Lq=1, Lkv=64)
+    assert f(s=dec, lwin=15) == _lib.HS_ERR_INVALID_ARG    # row 0 (position 63) sees keys 48 .. 63
+    assert f(s=dec, lwin=15, w=15, q=None) == _lib.HS_ERR_INVALID_ARG
+    assert f(w=0) == _lib.HS_ERR_INVALID_ARG
+    assert f(q=None) == _lib.HS_ERR_INVALID_ARG
+    assert f(wsb=0) == _lib.HS_ERR_WORKSPACE
+    assert f(s=dec, lwin=16, wsb=0) == _lib.HS_ERR_WORKSPACE   # long enough: checks go on to the workspace
+
+
 def test_block_rejects(L):
     s = shape()
     wsb = ws_size(L, s, n_sparse=2)

@@ -92,3 +92,43 @@ def test_sample_rows():
     for r in list(range(16)) + list(range(4080, 4096)) + [1022, 1023, 1024, 1025, 126, 127, 128, 129]:
         assert r in rows
     assert gen.sample_rows(4096, 1024, 128, n_random=50, seed=0, edge=16) == rows
+
+
+def test_window_kv_and_index_sets():
+    w = gen.Workload("t", 2, 50, 300, 8, 2, 128, "bf16", 40, 64, 1, "shifted")
+    kw, vw = gen.make_window_kv(w, 113, seed=1)
+    assert kw.shape == (2, 113, 2, 128) and vw.shape == kw.shape and kw.dtype == torch.bfloat16
+    kw2, _ = gen.make_window_kv(w, 113, seed=1)
+    assert torch.equal(kw, kw2)
+    assert abs(float(kw.float().std()) * math.sqrt(128) - 1.0) < 0.05     # std 1/sqrt(d)
+    # drawn apart from the block's other inputs: those are unchanged
+    a = gen.make_inputs(w, seed=1)
+    gen.make_window_kv(w, 113, seed=1)
+    assert torch.equal(a["k"], gen.make_inputs(w, seed=1)["k"])
+    for Lq, Lkv, topk in ((50, 300, 40), (3, 20000, 64)):
+        idx = gen.random_index_sets(2, 2, Lq, Lkv, topk, seed=7)
+        assert idx.dtype == torch.int32 and idx.shape == (2, 2, Lq, topk)
+        assert torch.equal(idx, gen.random_index_sets(2, 2, Lq, Lkv, topk, seed=7))
+        for b in range(2):
+            for h in range(2):
+                for i in range(Lq):
+                    pos = Lkv - Lq + i
+                    row = idx[b, h, i].tolist()
+                    take = min(pos + 1, topk)
+                    assert all(x == -1 for x in row[take:])
+                    sel = row[:take]
+                    assert all(0 <= x <= pos for x in sel) and sel == sorted(set(sel))
+
+
+def test_kv_cache_bytes():
+    import hybrid_sparse_attention_tcgen05_b200 as hs
+    B, Lkv, Hkv, d, n, win = 2, 1000, 4, 128, 3, 128
+    full = torch.empty(2, B, Lkv, Hkv, d, dtype=torch.bfloat16)
+    ring = torch.empty(n, 2, B, win, Hkv, d, dtype=torch.bfloat16)
+    r = hs.kv_cache_bytes(B, Lkv, Hkv, d, 2, n, win)
+    assert r["full"] == full.nbytes and r["sparse"] == 0 and r["dense_equivalent"] == (1 + n) * full.nbytes
+    r = hs.kv_cache_bytes(B, Lkv, Hkv, d, 2, n, win, own_window=True)
+    assert r["sparse"] == ring.nbytes and r["total"] == full.nbytes + ring.nbytes
+    # a prefill chunk of 64 rows needs window - 1 + 64 rows; never more than the cache
+    assert hs.kv_cache_bytes(B, Lkv, Hkv, d, 2, n, win, True, Lq=64)["sparse"] == n * 2 * B * 191 * Hkv * d * 2
+    assert hs.kv_cache_bytes(B, 100, Hkv, d, 2, n, win, True, Lq=100)["sparse"] == n * 2 * B * 100 * Hkv * d * 2
