@@ -145,26 +145,13 @@ __device__ __forceinline__ void find_bin(TopkShared &sh, const unsigned int *his
     }
 }
 
+// The exact select of one row by one CTA of NT threads (n > topk): a max /
+// min pass (copying the row to row_cache when SMEM), digit passes, and the
+// ordered compaction into o.  Every thread of the CTA calls it.
 template <bool SMEM>
-__global__ void __launch_bounds__(NT, 4)
-topk_radix_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv, int Hkv, int row_begin,
-                  int row_count, int r_lo, int topk, int32_t *__restrict__ idx, const int32_t *__restrict__ kv_len) {
-    extern __shared__ __align__(16) unsigned int row_cache[];
-    __shared__ TopkShared sh;
-    __shared__ int cnt_gt[NW], cnt_eq[NW];
-
-    const int r = r_lo + blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int i = row_begin + r;
-    const int n = row_keys(kv_len, b, Lq, Lkv, i);
-    const unsigned int *gu =
-        reinterpret_cast<const unsigned int *>(scores + (((size_t)b * Hkv + g) * row_count + r) * ld);
-    int32_t *o = idx + (((size_t)b * Hkv + g) * Lq + i) * (size_t)topk;
-
-    if (n <= topk) {
-        for (int t = tid; t < topk; t += NT) o[t] = t < n ? t : -1;
-        return;
-    }
+__device__ __forceinline__ void radix_select_row(TopkShared &sh, int *cnt_gt, int *cnt_eq, const unsigned int *gu,
+                                                 unsigned int *row_cache, int n, int topk, int32_t *o, int tid) {
+    const int lane = tid & 31, warp = tid >> 5;
     const bool aligned = (reinterpret_cast<uintptr_t>(gu) & 15u) == 0;
     for (int t = tid; t < 2 * kBins; t += NT) (&sh.h[0][0])[t] = 0u;
 
@@ -301,6 +288,29 @@ topk_radix_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lk
         gt_base += (int)(tot >> 16);
         eq_base += (int)(tot & 0xffffu);
     }
+}
+
+template <bool SMEM>
+__global__ void __launch_bounds__(NT, 4)
+topk_radix_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv, int Hkv, int row_begin,
+                  int row_count, int r_lo, int topk, int32_t *__restrict__ idx, const int32_t *__restrict__ kv_len) {
+    extern __shared__ __align__(16) unsigned int row_cache[];
+    __shared__ TopkShared sh;
+    __shared__ int cnt_gt[NW], cnt_eq[NW];
+
+    const int r = r_lo + blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x;
+    const int i = row_begin + r;
+    const int n = row_keys(kv_len, b, Lq, Lkv, i);
+    const unsigned int *gu =
+        reinterpret_cast<const unsigned int *>(scores + (((size_t)b * Hkv + g) * row_count + r) * ld);
+    int32_t *o = idx + (((size_t)b * Hkv + g) * Lq + i) * (size_t)topk;
+
+    if (n <= topk) {
+        for (int t = tid; t < topk; t += NT) o[t] = t < n ? t : -1;
+        return;
+    }
+    radix_select_row<SMEM>(sh, cnt_gt, cnt_eq, gu, row_cache, n, topk, o, tid);
 }
 
 // ------------------------------------------------------------ one warp per row
@@ -744,7 +754,358 @@ topk_warp_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv
         for (int w = 4 * ((n4 + 32) / 32) + lane; w < W; w += 32) mrow[w] = 0u;
 }
 
+// ------------------------------------------------ sampled single-pass select
+//
+// One CTA (NT threads) per (row, KV head), one pass over the row in the
+// common case.  A sample of SP_SAMPLE keys (SP_LINES lines of 32 consecutive
+// keys, evenly spaced over the row) brackets the k-th largest key: with
+// p = topk / n, the number of sampled keys above the k-th key is binomial
+// with mean SP_SAMPLE p and spread sigma = sqrt(SP_SAMPLE p (1 - p)), so the
+// sample's ranks SP_SAMPLE p -/+ SP_Z sigma give an interval [yA, yB] of
+// y = Ms - x (Ms: the sample's largest pattern) that holds the k-th key
+// unless the sample is off by more than SP_Z sigma.  One pass over the row
+// then sorts every key into: above the interval (taken: a bit in a shared-
+// memory bitmask), inside it (a candidate: listed with y - yA, and counted
+// in a 1024-bin histogram over the interval) or below it (not taken).  When
+// fewer than topk keys were taken and the candidates reach topk, the k-th
+// key is a candidate: the histogram names its bin, the few candidates in
+// that bin give its exact pattern, and the candidates below it plus the
+// lowest-indexed ones equal to it join the bitmask.  One compaction turns
+// the bitmask into the ascending index list (and, when asked, the dense
+// path's selection mask is the bitmask itself).  Otherwise (the interval
+// missed the k-th key, the candidate list overflowed, or the k-th key's bin
+// is crowded) the CTA runs the exact digit-pass select over the row.
+// Integer work throughout: the result is the exact top-k with ties to the
+// lower index, as every other select here computes it.
+constexpr int SP_LINES = 32;
+constexpr int SP_SAMPLE = SP_LINES * 32;
+constexpr float SP_Z = 3.0f;
+constexpr int SP_BINS = 1024;
+constexpr int SP_VARS = 64;                // words of SpVars, rounded up
+constexpr int SP_SMALL = SP_BINS / 2;      // candidates of the k-th key's bin held for the exact search
+constexpr int SP_MIN_KEYS = 64;            // shorter rows take the exact select directly
+constexpr int SP_UNROLL = 4;               // 16-byte loads in flight per thread in the pass
+
+struct SpVars {
+    unsigned int yA, yB, s1, ncand, nb, bstar, rb, fb, yT, keylim;
+    unsigned int wa[NW], wb[NW];
+};
+static_assert(sizeof(SpVars) <= SP_VARS * 4, "SpVars");
+
+// Shared-memory words before the bitmask: the histogram, the variables and
+// the candidate list (key, y - yA), or the exact select's state.
+__host__ __device__ constexpr int sp_region_words(int cap) {
+    const int a = SP_BINS + SP_VARS + 2 * cap;
+    const int b = (int)((sizeof(TopkShared) + 2 * NW * sizeof(int) + 3) / 4);
+    return ((a > b ? a : b) + 3) & ~3;
+}
+
+// Exclusive prefix over the CTA of one value per thread (via V.wa).
+__device__ __forceinline__ unsigned int sp_block_excl(SpVars &V, unsigned int v, int lane, int warp,
+                                                      unsigned int &total) {
+    unsigned int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const unsigned int y = __shfl_up_sync(FULL, incl, off);
+        if (lane >= off) incl += y;
+    }
+    if (lane == 31) V.wa[warp] = incl;
+    __syncthreads();
+    const unsigned int wv = lane < NW ? V.wa[lane] : 0u;
+    const unsigned int woff = __reduce_add_sync(FULL, lane < warp ? wv : 0u);
+    total = __reduce_add_sync(FULL, wv);
+    return woff + incl - v;
+}
+
+template <bool AL>
+__global__ void __launch_bounds__(NT, 2)
+topk_sampled_kernel(const float *__restrict__ scores, long long ld, int Lq, int Lkv, int Hkv, int row_begin,
+                    int row_count, int topk, int cap, int32_t *__restrict__ idx, uint32_t *__restrict__ mask,
+                    int W, const int32_t *__restrict__ kv_len) {
+    extern __shared__ __align__(16) unsigned int sp_smem[];
+    unsigned int *hist = sp_smem;
+    SpVars &V = *reinterpret_cast<SpVars *>(sp_smem + SP_BINS);
+    unsigned int *ck = sp_smem + SP_BINS + SP_VARS, *cy = ck + cap;
+    unsigned int *sel = sp_smem + sp_region_words(cap);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    // longest rows first; (batch, KV head) slowest
+    const long long item = blockIdx.x;
+    const int r = row_count - 1 - (int)(item % row_count);
+    const long long bg = item / row_count;
+    const int i = row_begin + r;
+    const int n = row_keys(kv_len, (int)(bg / Hkv), Lq, Lkv, i);
+    const unsigned int *u = reinterpret_cast<const unsigned int *>(scores + ((size_t)bg * row_count + r) * ld);
+    int32_t *o = idx + ((size_t)bg * Lq + i) * (size_t)topk;
+    uint32_t *mrow = mask ? mask + ((size_t)bg * Lq + i) * (size_t)W : nullptr;
+    if (n <= topk) {
+        for (int t = tid; t < topk; t += NT) o[t] = t < n ? t : -1;
+        if (mrow)
+            for (int w = tid; w < W; w += NT) {
+                const int lo = 32 * w;
+                mrow[w] = lo + 32 <= n ? FULL : (lo < n ? (1u << (n - lo)) - 1u : 0u);
+            }
+        return;
+    }
+    const int Wn = (n + 31) >> 5;
+    for (int t = tid; t < SP_BINS; t += NT) hist[t] = 0u;
+    for (int t = tid; t < Wn; t += NT) sel[t] = 0u;
+    if (tid == 0) {
+        V.ncand = 0u;
+        V.nb = 0u;
+    }
+
+    // the sample: lines q and q + 16 (warp q), one key per lane each
+    bool fb = n < SP_MIN_KEYS;
+    unsigned int x0 = 0u, x1 = 0u;
+    if (!fb) {
+        const long long span = n - 32;
+        x0 = __ldg(u + (int)(span * warp / (SP_LINES - 1)) + lane);
+        x1 = __ldg(u + (int)(span * (warp + NW) / (SP_LINES - 1)) + lane);
+    }
+    {
+        const unsigned int mx = __reduce_max_sync(FULL, max(x0, x1)), mn = __reduce_min_sync(FULL, min(x0, x1));
+        if (lane == 0) {
+            V.wa[warp] = mx;
+            V.wb[warp] = mn;
+        }
+    }
+    __syncthreads();
+    const unsigned int Ms = __reduce_max_sync(FULL, lane < NW ? V.wa[lane] : 0u);
+    const unsigned int ms = __reduce_min_sync(FULL, lane < NW ? V.wb[lane] : FULL);
+    fb = fb || Ms == ms;
+    const int s0 = max(0, (Ms > ms ? 32 - __clz(Ms - ms) : 0) - 10);
+    if (!fb) {
+        atomicAdd(&hist[(Ms - x0) >> s0], 1u);
+        atomicAdd(&hist[(Ms - x1) >> s0], 1u);
+    }
+    __syncthreads();
+    if (!fb && warp == 0) {
+        const float p = (float)topk / (float)n;
+        const float c = (float)SP_SAMPLE * p, sd = sqrtf((float)SP_SAMPLE * p * (1.f - p));
+        const int rh = (int)floorf(c - SP_Z * sd), rl = (int)ceilf(c + SP_Z * sd);
+        unsigned int yA = 0u, yB = FULL, rem, cnt;
+        if (rh >= 1) yA = wk_find(hist, (unsigned int)rh, lane, rem, cnt) << s0;
+        if (rl <= SP_SAMPLE) yB = ((wk_find(hist, (unsigned int)rl, lane, rem, cnt) + 1u) << s0) - 1u;
+        const unsigned int span = min(yB, Ms) - yA;   // y = Ms - x never exceeds Ms
+        if (lane == 0) {
+            V.yA = yA;
+            V.yB = yB;
+            V.s1 = (unsigned int)max(0, (span ? 32 - __clz(span) : 0) - 10);
+        }
+    }
+    __syncthreads();
+    const unsigned int yA = V.yA, yB = V.yB;
+    const int s1 = (int)V.s1;
+    for (int t = tid; t < SP_BINS; t += NT) hist[t] = 0u;
+    __syncthreads();
+
+    // the pass: warp w takes 128-key groups w, w + NW, ... (lane l: keys
+    // 4j .. 4j+3, j = 32 group + l), SP_UNROLL groups' loads in flight per
+    // lane; the group after the last full one carries the n mod 4 tail keys
+    if (!fb) {
+        const int n4 = n >> 2, nt = n & 3;
+        const unsigned int lt = (1u << lane) - 1u;
+        for (int jb = warp * 32; jb < n4 + 1; jb += NT * SP_UNROLL) {
+            uint4 vq[SP_UNROLL];
+#pragma unroll
+            for (int q = 0; q < SP_UNROLL; ++q) {
+                const int j = jb + q * NT + lane;
+                vq[q] = j < n4 ? ld4<AL>(u, j) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int q = 0; q < SP_UNROLL; ++q) {
+                const int j0 = jb + q * NT;
+                if (j0 >= n4 + 1) break;   // warp-uniform
+                const int j = j0 + lane;
+                unsigned int x[4];
+                bool ok[4];
+                if (j < n4) {
+                    x[0] = vq[q].x; x[1] = vq[q].y; x[2] = vq[q].z; x[3] = vq[q].w;
+                    ok[0] = ok[1] = ok[2] = ok[3] = true;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        ok[c] = j == n4 && c < nt;
+                        x[c] = ok[c] ? __ldg(u + 4 * n4 + c) : 0u;
+                    }
+                }
+                bool df[4], cd[4];
+                unsigned int yv[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const unsigned int y = Ms - x[c];
+                    df[c] = ok[c] && (x[c] > Ms || y < yA);
+                    cd[c] = ok[c] && x[c] <= Ms && y >= yA && y <= yB;
+                    yv[c] = y - yA;
+                }
+                // definites: word j >> 3 holds the nibbles of lanes 8m .. 8m+7
+                unsigned int wd = ((df[0] ? 1u : 0u) | (df[1] ? 2u : 0u) | (df[2] ? 4u : 0u) | (df[3] ? 8u : 0u))
+                                  << (4 * (lane & 7));
+                wd |= __shfl_xor_sync(FULL, wd, 1);
+                wd |= __shfl_xor_sync(FULL, wd, 2);
+                wd |= __shfl_xor_sync(FULL, wd, 4);
+                if ((lane & 7) == 0 && (j >> 3) < Wn) sel[j >> 3] = wd;
+                if (__any_sync(FULL, cd[0] || cd[1] || cd[2] || cd[3])) {
+                    int cbef = 0, ctot = 0;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const unsigned int bb = __ballot_sync(FULL, cd[c]);
+                        cbef += __popc(bb & lt);
+                        ctot += __popc(bb);
+                    }
+                    unsigned int base = 0u;
+                    if (lane == 0) base = atomicAdd(&V.ncand, (unsigned int)ctot);
+                    unsigned int at = __shfl_sync(FULL, base, 0) + (unsigned int)cbef;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        if (cd[c]) {
+                            if (at < (unsigned int)cap) {
+                                ck[at] = (unsigned int)(4 * j + c);
+                                cy[at] = yv[c];
+                            }
+                            atomicAdd(&hist[yv[c] >> s1], 1u);
+                            ++at;
+                        }
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    // keys taken so far (D) and the rank of the k-th key among the candidates
+    unsigned int dcnt = 0u;
+    for (int t = tid; t < Wn; t += NT) dcnt += __popc(sel[t]);
+    dcnt = __reduce_add_sync(FULL, dcnt);
+    if (lane == 0) V.wa[warp] = dcnt;
+    __syncthreads();
+    const unsigned int D = __reduce_add_sync(FULL, lane < NW ? V.wa[lane] : 0u);
+    const unsigned int ncand = V.ncand;
+    fb = fb || D >= (unsigned int)topk || D + ncand < (unsigned int)topk || ncand > (unsigned int)cap;
+    const unsigned int R = (unsigned int)topk - D;   // 1 .. ncand when !fb
+    __syncthreads();
+    if (!fb && warp == 0) {
+        unsigned int rb, cnt;
+        const unsigned int b = wk_find(hist, R, lane, rb, cnt);
+        if (lane == 0) {
+            V.bstar = b;
+            V.rb = rb;
+            V.fb = cnt > (unsigned int)SP_SMALL ? 1u : 0u;
+        }
+    }
+    __syncthreads();
+    fb = fb || V.fb != 0u;
+    __syncthreads();   // every thread has read the flag before the fallback's state overlays it
+    if (!fb) {
+        // the k-th key's bin: its candidates, (key, low bits of y - yA), into
+        // the histogram's space
+        const unsigned int bstar = V.bstar, lowm = s1 ? (1u << s1) - 1u : 0u;
+        for (int t = tid; t < (int)ncand; t += NT) {
+            const unsigned int yc = cy[t];
+            if ((yc >> s1) == bstar) {
+                const unsigned int slot = atomicAdd(&V.nb, 1u);
+                hist[2 * slot] = ck[t];
+                hist[2 * slot + 1] = yc & lowm;
+            }
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // the rb-th smallest low bits, bit by bit from the top: `ans`
+            // keeps the largest value with fewer than rb entries below it
+            const int nb = (int)V.nb;
+            const unsigned int rb = V.rb;
+            unsigned int ans = 0u;
+            for (int bit = s1 - 1; bit >= 0; --bit) {
+                const unsigned int t = ans | (1u << bit);
+                unsigned int c = 0u;
+                for (int e = lane; e < nb; e += 32) c += hist[2 * e + 1] < t;
+                if (__reduce_add_sync(FULL, c) < rb) ans = t;
+            }
+            unsigned int nl = 0u, ne = 0u;
+            for (int e = lane; e < nb; e += 32) {
+                nl += hist[2 * e + 1] < ans;
+                ne += hist[2 * e + 1] == ans;
+            }
+            const unsigned int take_eq = rb - __reduce_add_sync(FULL, nl);
+            ne = __reduce_add_sync(FULL, ne);
+            unsigned int keylim = FULL;
+            if (take_eq < ne) {
+                // the take_eq-th smallest key among the entries equal to ans
+                unsigned int kk = 0u;
+                for (int bit = 31 - __clz((unsigned int)n); bit >= 0; --bit) {
+                    const unsigned int t = kk | (1u << bit);
+                    unsigned int c = 0u;
+                    for (int e = lane; e < nb; e += 32) c += hist[2 * e + 1] == ans && hist[2 * e] < t;
+                    if (__reduce_add_sync(FULL, c) < take_eq) kk = t;
+                }
+                keylim = kk;
+            }
+            if (lane == 0) {
+                V.yT = (bstar << s1) | ans;
+                V.keylim = keylim;
+            }
+        }
+        __syncthreads();
+        const unsigned int yT = V.yT, keylim = V.keylim;
+        for (int t = tid; t < (int)ncand; t += NT) {
+            const unsigned int yc = cy[t], key = ck[t];
+            if (yc < yT || (yc == yT && key <= keylim)) atomicOr(&sel[key >> 5], 1u << (key & 31u));
+        }
+    } else {
+        radix_select_row<false>(*reinterpret_cast<TopkShared *>(sp_smem),
+                                reinterpret_cast<int *>(sp_smem) + sizeof(TopkShared) / 4,
+                                reinterpret_cast<int *>(sp_smem) + sizeof(TopkShared) / 4 + NW, u, nullptr, n,
+                                topk, o, tid);
+        if (mrow == nullptr) return;
+        __syncthreads();
+        for (int t = tid; t < Wn; t += NT) sel[t] = 0u;
+        __syncthreads();
+        for (int t = tid; t < topk; t += NT) {
+            const int key = o[t];
+            atomicOr(&sel[key >> 5], 1u << (key & 31));
+        }
+    }
+    __syncthreads();
+
+    // ascending index list from the bitmask: thread t owns words
+    // [t per, t per + per), its slots follow the exclusive prefix
+    const int per = (Wn + NT - 1) / NT, w0 = tid * per;
+    unsigned int cnt = 0u;
+    for (int w = w0; w < min(w0 + per, Wn); ++w) cnt += __popc(sel[w]);
+    unsigned int total;
+    unsigned int pos = sp_block_excl(V, cnt, lane, warp, total);
+    if (!fb)
+        for (int w = w0; w < min(w0 + per, Wn); ++w) {
+            unsigned int bits = sel[w];
+            while (bits) {
+                const int bb = __ffs(bits) - 1;
+                if (pos < (unsigned int)topk) o[pos] = 32 * w + bb;
+                ++pos;
+                bits &= bits - 1u;
+            }
+        }
+    if (mrow)
+        for (int w = tid; w < W; w += NT) mrow[w] = w < Wn ? sel[w] : 0u;
+}
+
 }  // namespace
+
+// Candidate-list capacity of the sampled select for rows of up to n_max keys
+// (1.6 times the expected candidates of the longest row, plus the sample
+// histogram's rounding) and its shared memory; 0 when it does not fit.
+static int sp_capacity(long long n_max, int topk) {
+    if (n_max <= topk) return 512;
+    const double kk = topk, nn = (double)n_max;
+    const double cand = 1.6 * 2.0 * SP_Z * sqrt(kk * (nn - kk) / SP_SAMPLE) + nn / 128.0 + 256.0;
+    const long long cap = ((long long)cand + 255) & ~255ll;
+    return (int)std::max(512ll, std::min(cap, 16384ll));
+}
+static size_t sp_smem_bytes(long long n_max, int cap) {
+    const long long wsel = (((n_max + 31) >> 5) + 3) & ~3ll;
+    return 4 * ((size_t)sp_region_words(cap) + (size_t)wsel);
+}
+constexpr size_t kSpMaxSmem = 160 * 1024;
 
 cudaError_t topk_launch(const Shape &s, const float *scores, long long ld, int row_begin, int row_count,
                         int topk, int32_t *idx, cudaStream_t st, uint32_t *mask, int W, bool *mask_done) {
@@ -759,9 +1120,42 @@ cudaError_t topk_launch(const Shape &s, const float *scores, long long ld, int r
     const long long n_items = (long long)s.B * s.Hkv * row_count;
     const long long off = (long long)s.Lkv - s.Lq;
     const bool al = (reinterpret_cast<uintptr_t>(scores) & 15u) == 0 && (ld & 3) == 0;
-    // HYSPARSE_TOPK_PATH=warp|block forces one kernel (the tests run both)
+    // HYSPARSE_TOPK_PATH=sampled|warp|block forces one kernel (the tests run
+    // all three); the sampled single pass is the default where its shared
+    // memory fits
     const char *force = getenv("HYSPARSE_TOPK_PATH");
     const bool f_warp = force && strcmp(force, "warp") == 0, f_block = force && strcmp(force, "block") == 0;
+    const long long n_max = s.kv_len ? (long long)s.Lkv : off + row_begin + row_count;
+    const int cap = sp_capacity(n_max, topk);
+    const size_t sp_bytes = sp_smem_bytes(n_max, cap);
+    // the sampled select for launches with few rows (decode).  With many
+    // rows its fixed per-row work (serial phases of one warp while the CTA
+    // waits at barriers, ~14 K warp instructions a row) costs more than the
+    // one-warp-per-row kernel's extra passes: measured slower at 8 K to 64 K
+    // keys per row.
+    const bool f_sampled = force && strcmp(force, "sampled") == 0;
+    const bool sampled = f_sampled || (!f_warp && !f_block && n_items < kWarpMinItems);
+    if (sampled && sp_bytes <= kSpMaxSmem && n_items <= 0x7fffffffLL) {
+        static size_t sp_attr = 0;
+        if (sp_bytes > sp_attr) {
+            cudaError_t e = cudaFuncSetAttribute(topk_sampled_kernel<true>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSpMaxSmem);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(topk_sampled_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSpMaxSmem);
+            if (e != cudaSuccess) return e;
+            sp_attr = kSpMaxSmem;
+        }
+        if (al)
+            topk_sampled_kernel<true><<<(unsigned int)n_items, NT, sp_bytes, st>>>(
+                scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, topk, cap, idx, mask, W, s.kv_len);
+        else
+            topk_sampled_kernel<false><<<(unsigned int)n_items, NT, sp_bytes, st>>>(
+                scores, ld, s.Lq, s.Lkv, s.Hkv, row_begin, row_count, topk, cap, idx, mask, W, s.kv_len);
+        count_launch();
+        if (mask_done) *mask_done = mask != nullptr;
+        return cudaGetLastError();
+    }
     const bool many = f_warp || (!f_block && n_items >= kWarpMinItems);
     if (many) {
         const unsigned int grid = (unsigned int)((n_items + WK_WARPS - 1) / WK_WARPS);

@@ -155,13 +155,14 @@ TOPK_BUCKET_EDGES = (9984, 25600)
 @pytest.mark.parametrize("case", ["ties", "ties_unaligned", "all_equal", "zeros_and_denormals", "long_rows",
                                   "flat_narrow", "flat_long_unaligned", "many_rows_ties",
                                   "many_rows_ties_aligned", "rows_8192", "short_rows_between_long",
-                                  "clustered", "clustered_wide"]
+                                  "clustered", "clustered_wide", "unsampled_peaks", "uniform_8192"]
                          + [f"edge{e}" for e in TOPK_BUCKET_EDGES]
                          + [f"edge{e}_unaligned" for e in TOPK_BUCKET_EDGES])
-@pytest.mark.parametrize("kernel", ["block", "warp"])
+@pytest.mark.parametrize("kernel", ["sampled", "block", "warp"])
 def test_topk_synthetic_rows_bit_exact(case, kernel, monkeypatch):
     """Score rows built directly (not by the CUDA path), with exact ties,
-    through both top-k kernels (one CTA per row / one warp per row)."""
+    through every top-k kernel (sampled single pass / one CTA per row / one
+    warp per row)."""
     monkeypatch.setenv("HYSPARSE_TOPK_PATH", kernel)
     g = torch.Generator().manual_seed(7)
     B, Hkv, Lq, Lkv, k = 2, 3, 37, 300, 29
@@ -187,6 +188,10 @@ def test_topk_synthetic_rows_bit_exact(case, kernel, monkeypatch):
         B, Hkv, Lq, Lkv, k = 2, 2, 1500, 1500, 700
     elif case.startswith("clustered"):   # the k-th key's bin holds more keys than the candidate list
         B, Hkv, Lq, Lkv, k = 1, 2, 2100, 3000, 900
+    elif case == "unsampled_peaks":   # the largest keys all lie outside the sampled lines
+        B, Hkv, Lq, Lkv, k = 1, 2, 64, 3000, 200
+    elif case == "uniform_8192":      # distinct values: no ties, the sampled pass's common case
+        B, Hkv, Lq, Lkv, k = 1, 2, 300, 8192, 1000
     s = torch.rand(B, Hkv, Lq, Lkv, generator=g)
     if case in ("ties", "ties_unaligned"):
         s = torch.round(s * 16) / 16
@@ -207,6 +212,18 @@ def test_topk_synthetic_rows_bit_exact(case, kernel, monkeypatch):
         span = 2.0 ** (-15 if case == "clustered" else -10)
         c = 0.5 + span * torch.rand(s.shape, generator=g)
         s = torch.where(torch.rand(s.shape, generator=g) < 0.8, c, s)
+    elif case == "unsampled_peaks":
+        # the sampled select reads 32 lines of 32 keys starting at
+        # floor((n - 32) q / 31); 1.5 k keys outside them get values above 1
+        for i in range(Lq):
+            n = Lkv - Lq + i + 1
+            inside = torch.zeros(n, dtype=torch.bool)
+            for q in range(32):
+                st = (n - 32) * q // 31
+                inside[st:st + 32] = True
+            out = (~inside).nonzero().flatten()
+            pick = out[torch.randperm(out.numel(), generator=g)[:3 * k // 2]]
+            s[:, :, i, pick] += 1.0
     shape = hs.HsShape(B, Lq, Lkv, 4 * Hkv, Hkv, 128, 1, 0.0)
     idx = hs.topk(shape, s.to(DEV), k)
     n_valid = [Lkv - Lq + i + 1 for _ in range(B) for _ in range(Hkv) for i in range(Lq)]
@@ -214,7 +231,7 @@ def test_topk_synthetic_rows_bit_exact(case, kernel, monkeypatch):
     assert torch.equal(idx.cpu(), o_idx)
 
 
-@pytest.mark.parametrize("topk_path", ["warp", "block"])
+@pytest.mark.parametrize("topk_path", ["sampled", "warp", "block"])
 @pytest.mark.parametrize("Lkv", [1000, 8500])
 def test_block_selection_mask_matches_stages(topk_path, Lkv, monkeypatch):
     """hysparse_block on the dense sparse path: with the one-warp-per-row
