@@ -461,10 +461,12 @@ def bench_ours(args, w, ws_, rank, local):
 
     # enough steps that the pipeline's fill and drain (the first copy in
     # before any compute, the last compute and copy out after the last copy
-    # in) are a small share of the timed region: about 1.5 s of device time,
-    # 4 to 32 steps (ms_per_step is already the max over ranks, so every rank
-    # runs the same count)
-    e2e_steps = int(max(4, min(32, 1500.0 / max(ms_per_step, 1e-3))))
+    # in) are a small share of the timed region: about 6 s of device time,
+    # 4 to 64 steps (ms_per_step is already the max over ranks, so every rank
+    # runs the same count).  At moe64k one step's copies take ~0.2 s each way
+    # against 0.35 s of compute, so over 4 steps the fill and drain alone
+    # added a quarter to every step.
+    e2e_steps = int(max(4, min(64, 6000.0 / max(ms_per_step, 1e-3))))
     e2e_step(0)
     e2e_step(1)
     torch.cuda.synchronize()
