@@ -404,6 +404,40 @@ def bench_ours(args, w, ws_, rank, local):
             torch.cuda.synchronize()
             fwd_ms += e0.elapsed_time(e1) / args.steps
 
+    # ---- (--own-window) the sparse layers with their own window K/V: each
+    # layer keeps [B, Lwin, Hkv, d] window keys and values (Lwin = Lkv in
+    # prefill, where every position is projected; the window itself in
+    # decode, a ring of the last tokens), timed against the same layers on
+    # the shared cache, same index sets, L2 flushed before each timed pass
+    own_window = None
+    if getattr(args, "own_window", False):
+        lwin = w.Lkv if w.Lq > 1 else min(w.window, w.Lkv)
+        kvw = [gen.make_window_kv(w, lwin, seed=args.seed + 1000 + n, device=str(dev)) for n in range(w.n_sparse)]
+        t_own = t_shared = 0.0
+        for _ in range(args.steps):
+            for own in (True, False):
+                flush.fill_(1.0)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for n in range(w.n_sparse):
+                    kw_, vw_ = kvw[n] if own else (None, None)
+                    hs.sparse_attn(qs[n], k, v, idx, gates[n], w.window, out=outs[n], ws=ws_full,
+                                   k_win=kw_, v_win=vw_)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                if own:
+                    t_own += e0.elapsed_time(e1) / args.steps / max(1, w.n_sparse)
+                else:
+                    t_shared += e0.elapsed_time(e1) / args.steps / max(1, w.n_sparse)
+        if hs.workspace_status(ws_full) != 0:
+            raise RuntimeError("device status after the own-window layers")
+        own_window = {"lwin": lwin, "sparse_per_layer_ms": t_own, "shared_cache_per_layer_ms": t_shared,
+                      "window_kv_bytes_per_layer": 2 * kvw[0][0].numel() * kvw[0][0].element_size(),
+                      "api": "hybrid_sparse_attention_tcgen05_b200.sparse_attn(k_win=, v_win=) "
+                             "(hysparse_sparse_attn_own_window)"}
+        del kvw
+
     # ---- end to end through the public API with host buffers
     # Each step copies its inputs from pinned host memory, runs the block and
     # copies every output back.  Consecutive steps are pipelined the way a
@@ -650,6 +684,8 @@ def bench_ours(args, w, ws_, rank, local):
     }
     if w.Lq == 1:
         res["decode_step_us"] = ms_per_step * 1e3
+    if own_window is not None:
+        res["own_window"] = own_window
     res["_inputs"] = inp
     return res
 
@@ -946,7 +982,7 @@ def decode_summary(res, peaks):
                               "frac_of_hbm": sp["gbs"] / peaks["hbm_gbs"], "peak_gbs": peaks["hbm_gbs"],
                               "work": "(k_eff + w_eff) K and V rows per (sequence, kv head) + q, gate, "
                                       "out, idx"},
-            "roofline": res["roofline"]}
+            "roofline": res["roofline"], **({"own_window": res["own_window"]} if "own_window" in res else {})}
 
 
 def profile_stage(args, w):
@@ -996,6 +1032,8 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--row-chunk", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--own-window", action="store_true",
+                    help="also time the sparse layers on their own window K/V against the shared cache")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--varlen", action="store_true",
                     help="decode workloads: every sequence at its own cache length (hysparse_block_varlen)")
