@@ -259,6 +259,15 @@ def l2_served(w):
     return w.Lq > 1 and 2 * w.B * w.Lkv * w.d * esz <= 64 * 2 ** 20
 
 
+def causal_tiles(Lq, Lkv, block=128):
+    """128 x 128 tiles of the Lq x Lkv score matrix that hold at least one
+    causal pair (row i sees keys 0 .. Lkv - Lq + i): the tiles a dense causal
+    pass runs, the count behind the dense-or-gather estimate and the executed
+    FLOPs of the dense-masked sparse layer."""
+    off = Lkv - Lq
+    return sum((off + min(Lq, block * (t + 1)) - 1) // block + 1 for t in range((Lq + block - 1) // block))
+
+
 def sparse_path_is_dense(w):
     """The library's choice between the dense-masked and the gather sparse
     kernel (same estimate as hysparse_api.cu; HYSPARSE_SPARSE_PATH overrides)."""
@@ -267,8 +276,7 @@ def sparse_path_is_dense(w):
         return False
     if env in ("dense", "gather"):
         return env == "dense"
-    off = w.Lkv - w.Lq
-    tiles = sum(int((off + min(w.Lq, 128 * (t + 1)) - 1) // 128) + 1 for t in range((w.Lq + 127) // 128))
+    tiles = causal_tiles(w.Lq, w.Lkv)
     per_tile = 2600.0 if (w.Hq // w.Hkv) % 2 == 0 else 4000.0
     dense_s = tiles * w.Hq * w.B * per_tile / (148.0 * 1.9e9)
     gather_s = (sum_min(w, w.topk) + sum_min(w, w.window)) * w.Hkv * w.B * 512.0 / 12.0e12
