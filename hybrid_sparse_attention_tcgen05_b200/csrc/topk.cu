@@ -15,11 +15,20 @@
 // "largest scores, ties to the lower index", already in ascending key order.
 // Integer work only: the result is exact and deterministic.
 //
-// One CTA of 512 threads per (row, KV head).  The max / min pass copies the
-// row into shared memory when it is short enough to keep four CTAs on an SM;
-// longer rows are re-read from global memory (L2) by every pass, which
-// measured faster than a shared-memory copy at lower occupancy.  Keys are
-// read four at a time (16 bytes); histogram bins take plain shared atomics.
+// Three kernels compute this same select:
+//   topk_warp_kernel     one warp per (row, KV head), for launches with many
+//                        rows (prefill);
+//   topk_sampled_kernel  one 512-thread CTA per row that brackets the k-th key
+//                        from a sample and settles it in one pass over the row
+//                        (launches with few rows: decode), falling back in
+//                        place to the exact CTA select below;
+//   topk_radix_kernel    the exact CTA select on its own (when forced, or for
+//                        few rows too long for the sampled kernel's shared
+//                        memory).
+// In the CTA select the max / min pass copies the row into shared memory
+// when it is short enough to keep four CTAs on an SM; longer rows are
+// re-read from global memory (L2) by every pass.  Keys are read four at a
+// time (16 bytes); histogram bins take plain shared atomics.
 #include <cstdlib>
 #include <cstring>
 
