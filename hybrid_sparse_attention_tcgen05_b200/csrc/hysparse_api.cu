@@ -160,6 +160,20 @@ bool use_gather_tc(const Shape &s) {
     return false;
 }
 
+// Whether hysparse_block runs its sparse layers as one gather launch (the
+// warp-MMA gather, several layers): by default for decode, where each layer
+// reads its rows from HBM and a lone layer fills half the SMs; prefill's
+// gather is served from L2 and bound by its instruction chains.
+// HYSPARSE_LAYER_GROUP=0|1 turns it off or on for every shape.
+bool group_sparse_layers(const Shape &s, int topk, int window, int n_sparse) {
+    if (n_sparse < 2 || s.k_win != nullptr || !sparse_mma_supported(s)) return false;
+    if (prefer_dense_sparse(s, topk, window) || use_gather_tc(s)) return false;
+    const char *e = getenv("HYSPARSE_LAYER_GROUP");
+    if (e && strcmp(e, "0") == 0) return false;
+    if (e && strcmp(e, "1") == 0) return true;
+    return s.Lq == 1;
+}
+
 // mask_ready: the dense path's selection bitmask in `ws` was already built
 // from this very index set (hysparse_block builds it once for all its layers).
 int run_sparse(const Shape &s, const void *q, const void *k, const void *v, const int32_t *idx,
@@ -371,6 +385,19 @@ int block_impl(const hs_shape *shape, const int32_t *kv_len, const Paging &pg, c
         if (rc != HS_OK) return rc;
     }
     const bool mask_ready = dense;
+    if (group_sparse_layers(s, topk, window, n_sparse)) {
+        // the layers share the index set and the cache: one gather launch per
+        // group of up to 16, so that each item's rows are read once per group
+        for (int n0 = 0; n0 < n_sparse; n0 += 16) {
+            const int n = n_sparse - n0 < 16 ? n_sparse - n0 : 16;
+            rc = cuda_status(sparse_attn_mma_layers_launch(s, n, q_sparse + n0, k, v, idx, topk, gate_logit + n0,
+                                                           window, out_sparse + n0,
+                                                           reinterpret_cast<unsigned int *>(ws), wait_limit_ns(),
+                                                           st));
+            if (rc != HS_OK) return rc;
+        }
+        return HS_OK;
+    }
     for (int n = 0; n < n_sparse; ++n) {
         rc = run_sparse(s, q_sparse[n], k, v, idx, topk, gate_logit[n], window, out_sparse[n],
                         nullptr, nullptr, ws, st, mask_ready);

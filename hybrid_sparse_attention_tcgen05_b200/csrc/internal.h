@@ -56,6 +56,12 @@ cudaError_t full_attn_scores_tc_launch(const Shape &s, const void *q, const void
 
 // sparse_mma.cu (bf16, d = 128, G <= 16)
 bool sparse_mma_supported(const Shape &s);
+// n (<= 16) sparse layers over the same index set and cache in one gather
+// launch (layer l: q[l], gate[l], out[l]; device pointers in host arrays)
+cudaError_t sparse_attn_mma_layers_launch(const Shape &s, int n, const void *const *q, const void *k, const void *v,
+                                          const int32_t *idx, int topk, const float *const *gate, int window,
+                                          void *const *out, unsigned int *status, unsigned long long wait_ns,
+                                          cudaStream_t st);
 cudaError_t sparse_attn_mma_launch(const Shape &s, const void *q, const void *k, const void *v,
                                    const int32_t *idx, int topk, const float *gate, int window, void *out,
                                    void *og, void *ol, unsigned int *status, unsigned long long wait_ns,

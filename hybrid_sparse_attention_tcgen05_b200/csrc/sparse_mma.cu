@@ -96,6 +96,10 @@ struct Branch {
     }
 };
 
+// Sparse layers one launch may run together (hysparse_block's layers share
+// the index set and the cache).
+constexpr int kMaxLayerGroup = 16;
+
 struct SpParams {
     const __nv_bfloat16 *q, *k, *v;
     const int32_t *idx;
@@ -115,6 +119,15 @@ struct SpParams {
     // Lkv - Lwin) read by the window branch, or NULL: the shared cache
     const __nv_bfloat16 *kw = nullptr, *vw = nullptr;
     int Lwin = 0;
+    // n_layers > 1: that many sparse layers over the same index set and
+    // cache in one launch, layer l with queries ql[l], gates gl[l], output
+    // outl[l] (q, gate, out unused).  Warps take (item, layer) pairs, layer
+    // fastest, so the warps of one item gather the same K/V rows at about the
+    // same time and all but the first find them in L2.
+    int n_layers = 1;
+    const __nv_bfloat16 *ql[kMaxLayerGroup] = {};
+    const float *gl[kMaxLayerGroup] = {};
+    __nv_bfloat16 *outl[kMaxLayerGroup] = {};
 };
 
 // Cache length of sequence b: kv_len[b] when given (a value outside
@@ -355,12 +368,18 @@ __device__ __forceinline__ void run_branch(const WarpCtx &w, bool from_list, con
     br.finish();
 }
 
-template <int NB, int CK>
+template <int NB, int CK, bool LG>   // LG: a group of layers (n_layers > 1)
 __global__ void __launch_bounds__(SpSmem<NB, CK>::SW * 32, 1) sparse_attn_mma(const SpParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long item = (long long)blockIdx.x * SpSmem<NB, CK>::SW + warp;
-    if (item >= (long long)p.B * p.Lq * p.Hkv) return;   // whole warp leaves together
+    const int nl = LG ? p.n_layers : 1;
+    long long item = (long long)blockIdx.x * SpSmem<NB, CK>::SW + warp;
+    if (item >= (long long)p.B * p.Lq * p.Hkv * nl) return;   // whole warp leaves together
+    const int layer = LG ? (int)(item % nl) : 0;
+    if (LG) item /= nl;
+    const __nv_bfloat16 *qp = LG ? p.ql[layer] : p.q;
+    const float *gp = LG ? p.gl[layer] : p.gate;
+    __nv_bfloat16 *outp = LG ? p.outl[layer] : p.out;
     // KV head slowest, then batch, then row: neighbouring warps gather from
     // the same KV head's cache (which stays in L2) and have similar row lengths
     const int i = (int)(item % p.Lq);
@@ -377,7 +396,7 @@ __global__ void __launch_bounds__(SpSmem<NB, CK>::SW * 32, 1) sparse_attn_mma(co
     for (int e = lane; e < 8 * NB * 16; e += 32) {
         const int h = e >> 4, cc = e & 15;
         uint4 val = make_uint4(0, 0, 0, 0);
-        if (h < G) val = __ldg(reinterpret_cast<const uint4 *>(p.q + (qrow + h) * 128) + cc);
+        if (h < G) val = __ldg(reinterpret_cast<const uint4 *>(qp + (qrow + h) * 128) + cc);
         *reinterpret_cast<uint4 *>(qs + sw_off(h, cc)) = val;
     }
     __syncwarp();
@@ -427,7 +446,7 @@ __global__ void __launch_bounds__(SpSmem<NB, CK>::SW * 32, 1) sparse_attn_mma(co
     const size_t orow = qrow * 128;
 #pragma unroll 1
     for (int which = 0; which < 3; ++which) {
-        __nv_bfloat16 *dst = which == 0 ? p.out : (which == 1 ? p.out_g : p.out_l);
+        __nv_bfloat16 *dst = which == 0 ? outp : (which == 1 ? p.out_g : p.out_l);
         if (dst == nullptr) continue;
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
@@ -439,7 +458,7 @@ __global__ void __launch_bounds__(SpSmem<NB, CK>::SW * 32, 1) sparse_attn_mma(co
                 const float il = ll > 0.f ? 1.f / ll : 0.f;
                 float sg = 0.f;
                 if (h < G) {
-                    const float x = p.gate[((size_t)b * p.Lq + i) * p.Hq + (size_t)g * G + h];
+                    const float x = gp[((size_t)b * p.Lq + i) * p.Hq + (size_t)g * G + h];
                     sg = 1.0f / (1.0f + expf(-x));
                 }
                 const float wg = which == 0 ? sg * ig : (which == 1 ? ig : 0.f);
@@ -619,20 +638,20 @@ cudaError_t launch_decode(const DecParams &dp, float *lse, float *scores, long l
     return cudaGetLastError();
 }
 
-template <int NB, int CK>
+template <int NB, int CK, bool LG = false>
 cudaError_t launch_nb(const SpParams &p, cudaStream_t st) {
     using S = SpSmem<NB, CK>;
     static bool attr = false;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(sparse_attn_mma<NB, CK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(sparse_attn_mma<NB, CK, LG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)S::bytes);
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    const long long items = (long long)p.B * p.Lq * p.Hkv;
+    const long long items = (long long)p.B * p.Lq * p.Hkv * (LG ? p.n_layers : 1);
     const long long blocks = (items + S::SW - 1) / S::SW;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-    sparse_attn_mma<NB, CK><<<(unsigned)blocks, S::SW * 32, S::bytes, st>>>(p); count_launch();
+    sparse_attn_mma<NB, CK, LG><<<(unsigned)blocks, S::SW * 32, S::bytes, st>>>(p); count_launch();
     return cudaGetLastError();
 }
 
@@ -654,6 +673,25 @@ cudaError_t sparse_attn_mma_launch(const Shape &s, const void *q, const void *k,
     p.Lwin = s.Lwin;
     if (s.G() <= 8) return tc::launch_nb<1, 32>(p, st);
     return tc::launch_nb<2, 32>(p, st);
+}
+
+cudaError_t sparse_attn_mma_layers_launch(const Shape &s, int n, const void *const *q, const void *k, const void *v,
+                                          const int32_t *idx, int topk, const float *const *gate, int window,
+                                          void *const *out, unsigned int *status, unsigned long long wait_ns,
+                                          cudaStream_t st) {
+    if (n < 1 || n > tc::kMaxLayerGroup || s.k_win != nullptr) return cudaErrorInvalidValue;
+    tc::SpParams p{(const __nv_bfloat16 *)q[0], (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, idx, gate[0],
+                   (__nv_bfloat16 *)out[0], nullptr, nullptr, s.B, s.Lq, s.Lkv, s.Hq, s.Hkv, s.G(), topk, window,
+                   s.scale * kLog2e, status, wait_ns, s.kv_len, s.block_table, s.page_shift, s.max_pages,
+                   s.num_pages};
+    p.n_layers = n;
+    for (int l = 0; l < n; ++l) {
+        p.ql[l] = (const __nv_bfloat16 *)q[l];
+        p.gl[l] = gate[l];
+        p.outl[l] = (__nv_bfloat16 *)out[l];
+    }
+    if (s.G() <= 8) return tc::launch_nb<1, 32, true>(p, st);
+    return tc::launch_nb<2, 32, true>(p, st);
 }
 
 size_t decode_ws_bytes(const Shape &s) {
