@@ -174,7 +174,11 @@ int hysparse_sparse_attn_own_window(const hs_shape *shape, const void *q, const 
  * gate logits, all reusing k, v and the one index set.
  * q_sparse, gate_logit and out_sparse are HOST arrays of n_sparse DEVICE
  * pointers.  idx_out (nullable) receives the index set [B][Hkv][Lq][topk];
- * when NULL it is kept in `ws`.  Errors: as the calls it makes. */
+ * when NULL it is kept in `ws`.  In decode (Lq == 1) the sparse layers run
+ * as one gather launch per group of up to 16 (they share the index set and
+ * the cache, so each row is read once per group); the outputs are those of
+ * one hysparse_sparse_attn call per layer, bit for bit.
+ * Errors: as the calls it makes. */
 int hysparse_block(const hs_shape *shape, const void *q_full, const void *k, const void *v,
                    void *out_full, float *lse, int n_sparse, const void *const *q_sparse,
                    const float *const *gate_logit, void *const *out_sparse, int topk, int window,
