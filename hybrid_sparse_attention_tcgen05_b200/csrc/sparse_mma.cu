@@ -579,7 +579,7 @@ __global__ void __launch_bounds__(SpSmem<NB, CK>::SW * 32, 1) decode_full_mma(co
 
 // One CTA per (batch, KV head): merge the split-K partials of the G heads
 // into O and LSE, then write the importance row from the logit stash.
-__global__ void __launch_bounds__(256) decode_combine(const DecParams dp, float *lse, float *scores,
+__global__ void __launch_bounds__(256, 4) decode_combine(const DecParams dp, float *lse, float *scores,
                                                       long long ld_scores) {
     const SpParams &p = dp.sp;
     const int g = blockIdx.x, b = blockIdx.y;
@@ -611,7 +611,29 @@ __global__ void __launch_bounds__(256) decode_combine(const DecParams dp, float 
     const float *st = dp.stash + qrow * (size_t)p.Lkv;
     float *srow = scores + ((size_t)b * p.Hkv + g) * ld_scores;
     const int Lb = seq_len(p, b);
-    for (int j = threadIdx.x; j < Lb; j += blockDim.x) {
+    // four consecutive keys per thread through 16-byte loads and stores when
+    // the rows allow it (more bytes in flight: the pass reads the whole
+    // stash), the same arithmetic per key as the scalar loop for the rest
+    int j_done = 0;
+    if ((p.Lkv & 3) == 0 && (ld_scores & 3) == 0 && (reinterpret_cast<uintptr_t>(st) & 15u) == 0 &&
+        (reinterpret_cast<uintptr_t>(srow) & 15u) == 0) {
+        const int n4 = Lb >> 2;
+#pragma unroll 2
+        for (int j4 = threadIdx.x; j4 < n4; j4 += blockDim.x) {
+            float4 sc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int h = 0; h < G; ++h) {
+                const float4 x = __ldg(reinterpret_cast<const float4 *>(st + (size_t)h * p.Lkv) + j4);
+                const float m = s_m[h], il = s_il[h];
+                sc.x = fmaf(ex2f(x.x - m), il, sc.x);
+                sc.y = fmaf(ex2f(x.y - m), il, sc.y);
+                sc.z = fmaf(ex2f(x.z - m), il, sc.z);
+                sc.w = fmaf(ex2f(x.w - m), il, sc.w);
+            }
+            reinterpret_cast<float4 *>(srow)[j4] = sc;
+        }
+        j_done = 4 * n4;
+    }
+    for (int j = j_done + threadIdx.x; j < Lb; j += blockDim.x) {
         float sc = 0.f;
         for (int h = 0; h < G; ++h) sc = fmaf(ex2f(st[(size_t)h * p.Lkv + j] - s_m[h]), s_il[h], sc);
         srow[j] = sc;
