@@ -54,3 +54,11 @@ def test_prefill_layer_group_when_forced(monkeypatch):
     monkeypatch.setenv("HYSPARSE_SPARSE_PATH", "gather")
     w = gen.Workload("pre_group", 1, 700, 700, 32, 2, 128, "bf16", 100, 128, 3, "shifted")
     _block_vs_layers(w, seed=9)
+
+
+def test_decode_layer_group_full_size(monkeypatch):
+    """The decode workload itself (64 sequences, 32768-token caches, 32/8 heads,
+    top-k 2048, 3 sparse layers): the grouped launch that the bench times
+    equals the per-layer calls bit for bit."""
+    monkeypatch.delenv("HYSPARSE_LAYER_GROUP", raising=False)
+    _block_vs_layers(gen.workload("decode"), seed=10)
