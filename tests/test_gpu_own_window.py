@@ -71,6 +71,7 @@ CASES = [
     ("decode", 3, 1, 1000, 8, 2, 128, "bf16", 128, 128, 128),          # ring of exactly the window
     ("fp32_d64", 2, 150, 150, 4, 2, 64, "f32", 32, 48, None),
     ("fp32_tail", 1, 40, 300, 4, 1, 128, "f32", 32, 64, 103),
+    ("fp32_decode", 2, 1, 300, 8, 2, 64, "f32", 64, 48, 48),
 ]
 
 
@@ -116,3 +117,15 @@ def test_own_window_rejects_short_buffer():
     with pytest.raises(hs._lib.HysparseError) as e:
         _run(w, cpu, kw, vw, idx)
     assert e.value.status == hs._lib.HS_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("sparse_path", ["dense", "gather"], indirect=True)
+def test_own_window_full_size_prefill_sampled(sparse_path):
+    """The prefill8k workload (8192 tokens, 32/8 heads, top-k 1024) with a
+    whole-cache window buffer, on both sparse paths; sampled rows (both ends,
+    the top-k and window edges, random rows) against the oracle."""
+    w = gen.workload("prefill8k", n_sparse=1)
+    cpu, kw, vw, idx = _setup(w, w.Lkv, seed=31)
+    got = _run(w, cpu, kw, vw, idx)
+    rows = rows_for(w.B, w.Lq, gen.sample_rows(w.Lq, w.topk, w.window, n_random=128, seed=31))
+    _check(w, cpu, kw, vw, idx, rows, got, f"prefill8k_own/{sparse_path}")
