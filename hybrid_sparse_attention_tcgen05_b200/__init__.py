@@ -184,13 +184,20 @@ def block(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_sparse: Sequence[
           out_full: Optional[torch.Tensor] = None, out_sparse: Optional[List[torch.Tensor]] = None,
           idx: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
           ws: Optional[torch.Tensor] = None, scale: Optional[float] = None,
-          kv_len: Optional[torch.Tensor] = None):
+          kv_len: Optional[torch.Tensor] = None, k_win: Optional[Sequence[torch.Tensor]] = None,
+          v_win: Optional[Sequence[torch.Tensor]] = None):
     """One hybrid block.  Returns (out_full, lse, idx, [out_sparse_n]).
 
     kv_len (int32 [B] on the device, decode only): sequence b's cache is the
     first kv_len[b] rows of k[b] and v[b], its new query at position
-    kv_len[b] - 1 (hysparse_block_varlen)."""
-    dev = _need_cuda(q, k, v, out_full, idx, lse, ws, kv_len, *q_sparse, *gate_logit, *(out_sparse or []))
+    kv_len[b] - 1 (hysparse_block_varlen).
+
+    k_win, v_win (one [B, lwin, Hkv, d] tensor per sparse layer, the same
+    lwin for all): the layers' own window K/V for cache positions
+    Lkv - lwin .. Lkv - 1, read by their window branches
+    (hysparse_block_own_window)."""
+    dev = _need_cuda(q, k, v, out_full, idx, lse, ws, kv_len, *q_sparse, *gate_logit, *(out_sparse or []),
+                     *(k_win or []), *(v_win or []))
     s = shape_of(q, k, scale)
     n = len(q_sparse)
     if len(gate_logit) != n:
@@ -218,6 +225,23 @@ def block(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_sparse: Sequence[
             ctypes.cast(oa, ctypes.c_void_p), int(k_top), int(window), _ptr(idx),
             _ptr(ws), ws.numel(), _stream(dev))
         _lib.check(st, "hysparse_block_varlen")
+        return out_full, lse, idx, out_sparse
+    if k_win is not None or v_win is not None:
+        if k_win is None or v_win is None or len(k_win) != n or len(v_win) != n:
+            raise ValueError("one k_win and one v_win tensor per sparse layer")
+        lwin = k_win[0].shape[1] if n else 0
+        want = (k.shape[0], lwin) + tuple(k.shape[2:])
+        for t in (*k_win, *v_win):
+            if tuple(t.shape) != want or t.dtype != k.dtype:
+                raise TypeError("k_win and v_win must be [B, lwin, Hkv, d] of k's dtype, one lwin for all layers")
+        ka = PA(*[x.data_ptr() for x in k_win])
+        va = PA(*[x.data_ptr() for x in v_win])
+        st = _lib.lib().hysparse_block_own_window(
+            ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(out_full), _ptr(lse), n,
+            ctypes.cast(qa, ctypes.c_void_p), ctypes.cast(ga, ctypes.c_void_p), ctypes.cast(ka, ctypes.c_void_p),
+            ctypes.cast(va, ctypes.c_void_p), int(lwin), ctypes.cast(oa, ctypes.c_void_p), int(k_top),
+            int(window), _ptr(idx), int(row_chunk), _ptr(ws), ws.numel(), _stream(dev))
+        _lib.check(st, "hysparse_block_own_window")
         return out_full, lse, idx, out_sparse
     st = _lib.lib().hysparse_block(
         ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(out_full), _ptr(lse), n,

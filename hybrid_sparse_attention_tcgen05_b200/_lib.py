@@ -29,6 +29,7 @@ EXPORTS = (
     "hysparse_topk",
     "hysparse_sparse_attn",
     "hysparse_sparse_attn_own_window",
+    "hysparse_block_own_window",
     "hysparse_block",
     "hysparse_block_varlen",
     "hysparse_block_paged",
@@ -80,6 +81,8 @@ def lib():
     L.hysparse_sparse_attn_own_window.restype = I
     L.hysparse_block.argtypes = [SP, P, P, P, P, P, I, P, P, P, I, I, P, I, P, SZ, P]
     L.hysparse_block.restype = I
+    L.hysparse_block_own_window.argtypes = [SP, P, P, P, P, P, I, P, P, P, P, I, P, I, I, P, I, P, SZ, P]
+    L.hysparse_block_own_window.restype = I
     L.hysparse_block_varlen.argtypes = [SP, P, P, P, P, P, P, I, P, P, P, I, I, P, P, SZ, P]
     L.hysparse_block_varlen.restype = I
     L.hysparse_block_paged.argtypes = [SP, P, P, I, I, I, P, P, P, P, P, I, P, P, P, I, I, P, P, SZ, P]

@@ -317,12 +317,21 @@ struct Paging {
     int page_size = 0, max_pages = 0, num_pages = 0;
 };
 
+// The sparse layers' own window K/V (hysparse_block_own_window): layer n
+// reads k[n], v[n], lwin rows each.  k == NULL: the shared cache.
+struct OwnWindows {
+    const void *const *k = nullptr;
+    const void *const *v = nullptr;
+    int lwin = 0;
+};
+
 // hysparse_block; hysparse_block_varlen when kv_len is set; and
 // hysparse_block_paged when the paging table is set too
 int block_impl(const hs_shape *shape, const int32_t *kv_len, const Paging &pg, const void *q_full, const void *k,
                const void *v, void *out_full, float *lse, int n_sparse, const void *const *q_sparse,
                const float *const *gate_logit, void *const *out_sparse, int topk, int window,
-               int32_t *idx_out, int row_chunk, void *ws, size_t ws_bytes, hs_stream_t stream) {
+               int32_t *idx_out, int row_chunk, void *ws, size_t ws_bytes, hs_stream_t stream,
+               const OwnWindows &ow = OwnWindows{}) {
     Shape s;
     int rc = resolve_shape(shape, &s);
     if (rc != HS_OK) return rc;
@@ -355,6 +364,15 @@ int block_impl(const hs_shape *shape, const int32_t *kv_len, const Paging &pg, c
     for (int n = 0; n < n_sparse; ++n)
         if (!aligned16(q_sparse[n]) || !aligned16(gate_logit[n]) || !aligned16(out_sparse[n]))
             return HS_ERR_INVALID_ARG;
+    if (ow.k != nullptr) {
+        // own window buffers: fixed-length caches, every layer's buffer
+        // reaching back to the first row's window
+        if (kv_len != nullptr || ow.v == nullptr || ow.lwin < 1 || ow.lwin > s.Lkv) return HS_ERR_INVALID_ARG;
+        const int first_key = s.Lkv - s.Lq - window + 1 > 0 ? s.Lkv - s.Lq - window + 1 : 0;
+        if (s.Lkv - ow.lwin > first_key) return HS_ERR_INVALID_ARG;
+        for (int n = 0; n < n_sparse; ++n)
+            if (!aligned16(ow.k[n]) || !aligned16(ow.v[n])) return HS_ERR_INVALID_ARG;
+    }
     if (!aligned16(ws)) return HS_ERR_INVALID_ARG;
     const int chunk = (row_chunk <= 0 || row_chunk > s.Lq) ? s.Lq : row_chunk;
     const WsLayout L = ws_layout(s, topk, chunk);
@@ -385,6 +403,18 @@ int block_impl(const hs_shape *shape, const int32_t *kv_len, const Paging &pg, c
         if (rc != HS_OK) return rc;
     }
     const bool mask_ready = dense;
+    if (ow.k != nullptr) {
+        for (int n = 0; n < n_sparse; ++n) {
+            Shape sl = s;
+            sl.k_win = ow.k[n];
+            sl.v_win = ow.v[n];
+            sl.Lwin = ow.lwin;
+            rc = run_sparse(sl, q_sparse[n], k, v, idx, topk, gate_logit[n], window, out_sparse[n], nullptr,
+                            nullptr, ws, st, mask_ready);
+            if (rc != HS_OK) return rc;
+        }
+        return HS_OK;
+    }
     if (group_sparse_layers(s, topk, window, n_sparse)) {
         // the layers share the index set and the cache: one gather launch per
         // group of up to 16, so that each item's rows are read once per group
@@ -414,6 +444,20 @@ int hysparse_block(const hs_shape *shape, const void *q_full, const void *k, con
                    hs_stream_t stream) {
     return block_impl(shape, nullptr, Paging{}, q_full, k, v, out_full, lse, n_sparse, q_sparse, gate_logit,
                       out_sparse, topk, window, idx_out, row_chunk, ws, ws_bytes, stream);
+}
+
+int hysparse_block_own_window(const hs_shape *shape, const void *q_full, const void *k, const void *v,
+                              void *out_full, float *lse, int n_sparse, const void *const *q_sparse,
+                              const float *const *gate_logit, const void *const *k_win, const void *const *v_win,
+                              int lwin, void *const *out_sparse, int topk, int window, int32_t *idx_out,
+                              int row_chunk, void *ws, size_t ws_bytes, hs_stream_t stream) {
+    if (n_sparse > 0 && (k_win == nullptr || v_win == nullptr)) return HS_ERR_INVALID_ARG;
+    OwnWindows ow;
+    ow.k = n_sparse > 0 ? k_win : nullptr;
+    ow.v = v_win;
+    ow.lwin = lwin;
+    return block_impl(shape, nullptr, Paging{}, q_full, k, v, out_full, lse, n_sparse, q_sparse, gate_logit,
+                      out_sparse, topk, window, idx_out, row_chunk, ws, ws_bytes, stream, ow);
 }
 
 int hysparse_block_varlen(const hs_shape *shape, const int32_t *kv_len, const void *q_full, const void *k,

@@ -184,6 +184,22 @@ int hysparse_block(const hs_shape *shape, const void *q_full, const void *k, con
                    const float *const *gate_logit, void *const *out_sparse, int topk, int window,
                    int32_t *idx_out, int row_chunk, void *ws, size_t ws_bytes, hs_stream_t stream);
 
+/* hysparse_block with every sparse layer reading its window branch from its
+ * own window K/V (write-up section 2.2; the variant of
+ * hysparse_sparse_attn_own_window): k_win and v_win are HOST arrays of
+ * n_sparse DEVICE pointers, layer n's [B][lwin][Hkv][d] buffers for cache
+ * positions Lkv - lwin .. Lkv - 1 (layouts and limits as in
+ * hysparse_sparse_attn_own_window, the same lwin for every layer).  The full
+ * layer, the index set and the global branches are hysparse_block's; the
+ * outputs equal hysparse_sparse_attn_own_window per layer on the block's
+ * index set.  Fixed-length caches only.  Errors: as hysparse_block, and
+ * HS_ERR_INVALID_ARG for a missing, misaligned or too short window buffer. */
+int hysparse_block_own_window(const hs_shape *shape, const void *q_full, const void *k, const void *v,
+                              void *out_full, float *lse, int n_sparse, const void *const *q_sparse,
+                              const float *const *gate_logit, const void *const *k_win, const void *const *v_win,
+                              int lwin, void *const *out_sparse, int topk, int window, int32_t *idx_out,
+                              int row_chunk, void *ws, size_t ws_bytes, hs_stream_t stream);
+
 /* One decode step of the hybrid block over a batch whose sequences have
  * caches of different lengths (serving: every sequence decodes one token,
  * each at its own position).  Same computation, arguments and layouts as

@@ -178,6 +178,29 @@ def test_block_rejects(L):
     assert f(chunk=8, wsb=ws_size(L, s, n_sparse=2, row_chunk=8) - 1) == _lib.HS_ERR_WORKSPACE
 
 
+def test_block_own_window_rejects(L):
+    """hysparse_block_own_window: every layer's window buffer present, aligned
+    and reaching back to the first row's window, before anything runs."""
+    s = shape()            # Lq = Lkv = 64: lwin must be 64
+    wsb = ws_size(L, s, n_sparse=2)
+    PA = ctypes.c_void_p * 2
+    qa, ga, oa = PA(A, A + 256), PA(A + 512, A + 768), PA(A + 1024, A + 1280)
+    kw, vw = PA(A + 2048, A + 4096), PA(A + 6144, A + 8192)
+    c = lambda x: ctypes.cast(x, ctypes.c_void_p)
+
+    def f(**a):
+        return L.hysparse_block_own_window(ctypes.byref(s), P(1), P(2), P(3), P(4), None, 2, c(qa), c(ga),
+                                           a.get("kw", c(kw)), a.get("vw", c(vw)), a.get("lwin", 64), c(oa), 8,
+                                           16, None, 0, P(7), a.get("wsb", wsb), None)
+    assert f(kw=None) == _lib.HS_ERR_INVALID_ARG
+    assert f(vw=None) == _lib.HS_ERR_INVALID_ARG
+    assert f(lwin=63) == _lib.HS_ERR_INVALID_ARG      # row 0 sees key 0
+    assert f(lwin=65) == _lib.HS_ERR_INVALID_ARG
+    assert f(lwin=0) == _lib.HS_ERR_INVALID_ARG
+    assert f(kw=c(PA(A + 2048, A + 4100))) == _lib.HS_ERR_INVALID_ARG   # layer 1 misaligned
+    assert f(wsb=wsb - 1) == _lib.HS_ERR_WORKSPACE      # valid window buffers: on to the workspace check
+
+
 def test_block_varlen_rejects(L):
     """hysparse_block_varlen: decode shapes on the bf16 path only, a 4-byte
     aligned length array, and the workspace of the fixed-length block."""

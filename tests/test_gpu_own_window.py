@@ -129,3 +129,39 @@ def test_own_window_full_size_prefill_sampled(sparse_path):
     got = _run(w, cpu, kw, vw, idx)
     rows = rows_for(w.B, w.Lq, gen.sample_rows(w.Lq, w.topk, w.window, n_random=128, seed=31))
     _check(w, cpu, kw, vw, idx, rows, got, f"prefill8k_own/{sparse_path}")
+
+
+# (name, B, Lq, Lkv, Hq, Hkv, topk, window, lwin, n_sparse, sparse_path)
+BLOCK_CASES = [
+    ("prefill_dense", 1, 600, 600, 8, 2, 64, 128, 600, 3, "dense"),
+    ("prefill_gather", 1, 600, 600, 8, 2, 64, 128, 600, 3, "gather"),
+    ("prefill_auto_g3", 1, 400, 400, 6, 2, 64, 128, 400, 2, None),
+    ("chunk_tail", 2, 64, 1000, 8, 2, 96, 128, 191, 2, None),
+    ("decode_ring", 4, 1, 2000, 32, 8, 256, 128, 128, 3, None),
+]
+
+
+@pytest.mark.parametrize("case", BLOCK_CASES, ids=[c[0] for c in BLOCK_CASES])
+def test_block_own_window_equals_layer_calls(case, monkeypatch):
+    """hysparse_block_own_window: the full layer and index set of the plain
+    block, and every sparse layer equal to hysparse_sparse_attn_own_window on
+    that index set, bit for bit."""
+    name, B, Lq, Lkv, Hq, Hkv, topk, window, lwin, n_sparse, path = case
+    monkeypatch.delenv("HYSPARSE_SPARSE_PATH", raising=False)
+    if path is not None:
+        monkeypatch.setenv("HYSPARSE_SPARSE_PATH", path)
+    w = gen.Workload(name, B, Lq, Lkv, Hq, Hkv, 128, "bf16", topk, window, n_sparse,
+                     "shifted" if Lq > 1 else "normal")
+    inp = gen.make_inputs(w, seed=41, device=DEV)
+    wins = [gen.make_window_kv(w, lwin, seed=500 + n, device=DEV) for n in range(n_sparse)]
+    kw, vw = [x[0] for x in wins], [x[1] for x in wins]
+    of, lse, idx, outs = hs.block(inp["q"], inp["k"], inp["v"], inp["q_sparse"], inp["gate"], topk, window,
+                                  k_win=kw, v_win=vw)
+    pf, plse, pidx, _ = hs.block(inp["q"], inp["k"], inp["v"], inp["q_sparse"], inp["gate"], topk, window)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, pidx) and torch.equal(of, pf) and torch.equal(lse, plse)
+    for n in range(n_sparse):
+        ref = hs.sparse_attn(inp["q_sparse"][n], inp["k"], inp["v"], idx, inp["gate"][n], window,
+                             k_win=kw[n], v_win=vw[n])
+        torch.cuda.synchronize()
+        assert torch.equal(outs[n], ref), f"layer {n}"
