@@ -2,7 +2,7 @@
 (on the CPU, in a temporary directory) and check that at least one pin
 catches it.  This shows the pins constrain every step: causal bound, scale,
 max subtraction, group mapping, score accumulation, tie order, window extent,
-gate direction."""
+gate direction, and the own-window layer's buffer and row offset."""
 import os
 import shutil
 
@@ -25,6 +25,15 @@ MUTANTS = {
                      "out[o + c] = gs * ol[c] + (1.0 - gs) * og[c];"),
     "lse_without_log": ("return m + log(l);", "return m + l;"),
     "topk_keeps_k_minus_1": ("int take = n < topk ? n : topk;", "int take = n < topk ? n : topk - 1;"),
+    # the own-window layer's local branch reading the shared cache at the
+    # buffer's row numbers (in range, wrong values)
+    "own_window_reads_shared_cache": (
+        "attend_list(q, kw, vw, b, g, Lwin, Hkv, d, scale, keys_l, nl, s, ol, NULL);",
+        "attend_list(q, k, v, b, g, Lkv, Hkv, d, scale, keys_l, nl, s, ol, NULL);"),
+    # the own-window buffer's first row taken one position too late (every
+    # read stays inside the buffer: rows are validated before any is read)
+    "own_window_offset_plus_one": ("const int woff = kw ? Lkv - Lwin : 0;",
+                                   "const int woff = kw ? Lkv - Lwin + 1 : 0;"),
 }
 
 
