@@ -692,6 +692,13 @@ def bench_ours(args, w, ws_, rank, local):
     }
     if w.Lq == 1:
         res["decode_step_us"] = ms_per_step * 1e3
+        if w.dtype == "bf16" and w.n_sparse > 1 and os.environ.get("HYSPARSE_LAYER_GROUP") != "0":
+            # the stage loop times the sparse layers as single-layer calls;
+            # hysparse_block runs them as one grouped launch, whose time is the
+            # step less the other two stages
+            res["sparse_grouped_ms_est"] = max(0.0, ms_per_step - per["full"] - per["topk"])
+            res["stages_note"] = ("stages time each sparse layer as its own call; the block runs the "
+                                  "decode sparse layers as one grouped launch (sparse_grouped_ms_est)")
     if own_window is not None:
         res["own_window"] = own_window
     res["_inputs"] = inp
@@ -990,7 +997,9 @@ def decode_summary(res, peaks):
                               "frac_of_hbm": sp["gbs"] / peaks["hbm_gbs"], "peak_gbs": peaks["hbm_gbs"],
                               "work": "(k_eff + w_eff) K and V rows per (sequence, kv head) + q, gate, "
                                       "out, idx"},
-            "roofline": res["roofline"], **({"own_window": res["own_window"]} if "own_window" in res else {})}
+            "roofline": res["roofline"], **({"own_window": res["own_window"]} if "own_window" in res else {}),
+            **({"sparse_grouped_ms_est": res["sparse_grouped_ms_est"], "stages_note": res["stages_note"]}
+               if "sparse_grouped_ms_est" in res else {})}
 
 
 def profile_stage(args, w):
