@@ -25,6 +25,8 @@
  *   scores (one row chunk)             [B][Hkv][row_count][ld_scores] float
  *   idx                                [B][Hkv][Lq][topk] int32
  *   gate_logit                         [B][Lq][Hq]        float
+ *   k_win, v_win (own-window calls)    [B][lwin][Hkv][d]  (dtype of the shape),
+ *                                      row r = cache position Lkv - lwin + r
  *
  * Conventions for every entry point:
  *   - All device buffers are owned by the caller (e.g. allocated by PyTorch).
