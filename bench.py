@@ -259,6 +259,13 @@ def l2_served(w):
     return w.Lq > 1 and 2 * w.B * w.Lkv * w.d * esz <= 64 * 2 ** 20
 
 
+def e2e_step_count(ms_per_step):
+    """Steps of the end-to-end loop: about 6 s of device time, 4 to 64 steps,
+    so that the copy pipeline's fill and drain are a small share of it
+    (ms_per_step is the max over ranks, so every rank runs the same count)."""
+    return int(max(4, min(64, 6000.0 / max(ms_per_step, 1e-3))))
+
+
 def causal_tiles(Lq, Lkv, block=128):
     """128 x 128 tiles of the Lq x Lkv score matrix that hold at least one
     causal pair (row i sees keys 0 .. Lkv - Lq + i): the tiles a dense causal
@@ -569,7 +576,7 @@ def bench_ours(args, w, ws_, rank, local):
     # runs the same count).  At moe64k one step's copies take ~0.2 s each way
     # against 0.35 s of compute, so over 4 steps the fill and drain alone
     # added a quarter to every step.
-    e2e_steps = int(max(4, min(64, 6000.0 / max(ms_per_step, 1e-3))))
+    e2e_steps = e2e_step_count(ms_per_step)
     e2e_step(0)
     e2e_step(1)
     torch.cuda.synchronize()
@@ -829,7 +836,7 @@ def bench_varlen(args, w, ws_, rank, local):
         for a_, b_ in zip(h_res, [out, *outs]):
             a_.copy_(b_, non_blocking=True)
 
-    e2e_steps = int(max(4, min(32, 1500.0 / max(ms_per_step, 1e-3))))
+    e2e_steps = e2e_step_count(ms_per_step)
     e2e_step()
     torch.cuda.synchronize()
     if ws_ > 1:

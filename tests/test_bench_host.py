@@ -29,3 +29,11 @@ def test_comment_edit_keeps_code_and_code_edit_changes_it():
     assert bench.code_only(commented) == bench.code_only(CODE)
     assert bench.code_only(CODE.replace("1.f", "2.f")) != bench.code_only(CODE)
 
+
+
+def test_e2e_step_count():
+    # about 6 s of device time, 4 to 64 steps
+    assert bench.e2e_step_count(351.4) == 17
+    assert bench.e2e_step_count(1.6) == 64
+    assert bench.e2e_step_count(3000.0) == 4
+    assert bench.e2e_step_count(0.0) == 64
